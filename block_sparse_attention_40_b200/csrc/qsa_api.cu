@@ -1,0 +1,735 @@
+// qsa_api.cu -- C ABI of libqsa.so: argument checks, workspace layout, TMA descriptors and
+// kernel launches for QSA prefill, append and decode on sm_100a.  The declarations and the
+// contract of every entry point are in include/qsa.h.
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/qsa.h"
+#include "qsa_attn.cuh"
+#include "qsa_common.cuh"
+#include "qsa_misc.cuh"
+#include "qsa_score.cuh"
+
+using namespace qsa;
+
+namespace {
+
+constexpr int kVersion = 100;   // 0.1.0
+constexpr int kDefaultRowsPerTile = 8;
+constexpr int kDefaultScoreChunkRows = 4096;
+constexpr int kTopkSmemCap = 32768;     // row scores cached in shared memory up to this n_c
+constexpr int kNumSMsFallback = 148;
+
+// ---- driver entry point for tensor-map encoding (no link-time libcuda dependency) ----
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return kNumSMsFallback;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return kNumSMsFallback;
+  return n;
+}
+
+// bf16 tensor map, 128-byte swizzle, inner box of 64 elements (128 bytes).
+bool make_tmap(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+               const uint64_t* strides_bytes, const uint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gd[5];
+  cuuint64_t gs[4];
+  cuuint32_t bd[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bd[i] = box[i];
+    es[i] = 1;
+  }
+  for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gd, gs, bd,
+                  es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---- workspace carving ---------------------------------------------------------------
+struct Carver {
+  size_t off = QSA_WS_HEADER_BYTES;
+  size_t take(size_t bytes) {
+    const size_t o = off;
+    off = round_up(off + bytes, 256);
+    return o;
+  }
+};
+
+struct PrefillGeom {
+  int64_t T = 0;
+  int32_t max_len = 0;
+  int64_t total_blocks = 0;
+  int32_t max_nc = 0;
+  int64_t ld = 0;
+  int32_t score_tiles = 0;
+  int32_t attn_tiles = 0;
+  int32_t R = kDefaultRowsPerTile;
+  int32_t topk = 512;
+  int32_t chunk_rows = kDefaultScoreChunkRows;
+  PlanLayout pl;
+  int32_t max_words = 1;
+  // workspace offsets
+  size_t o_meta = 0, o_kbar = 0, o_nc = 0, o_scores = 0, o_idx = 0, o_cnt = 0, o_plan = 0, total = 0;
+};
+
+qsa_status prefill_geom(const int32_t* h_cu, int32_t num_seqs, const qsa_params& p,
+                        PrefillGeom* g) {
+  if (!h_cu || num_seqs <= 0) return QSA_ERR_INVALID_ARG;
+  if (p.topk_blocks < 1 || p.topk_blocks > QSA_MAX_TOPK) return QSA_ERR_INVALID_ARG;
+  if (h_cu[0] != 0) return QSA_ERR_INVALID_ARG;
+  g->R = p.rows_per_tile > 0 ? p.rows_per_tile : kDefaultRowsPerTile;
+  if (g->R < 1 || g->R > 10) return QSA_ERR_INVALID_ARG;
+  g->topk = p.topk_blocks;
+  g->chunk_rows = p.score_chunk_rows > 0 ? p.score_chunk_rows : kDefaultScoreChunkRows;
+  if (g->chunk_rows < 16) g->chunk_rows = 16;
+  int64_t T = 0, blocks = 0;
+  int32_t max_len = 0;
+  int64_t st = 0, at = 0;
+  for (int s = 0; s < num_seqs; ++s) {
+    const int64_t L = static_cast<int64_t>(h_cu[s + 1]) - h_cu[s];
+    if (L < 1 || L > QSA_MAX_SEQ_LEN) return QSA_ERR_INVALID_ARG;
+    T += L;
+    blocks += L / 4;
+    max_len = std::max<int32_t>(max_len, static_cast<int32_t>(L));
+    st += (L + 15) / 16;
+    at += (L + g->R - 1) / g->R;
+  }
+  if (T > (int64_t(1) << 26)) return QSA_ERR_UNSUPPORTED;
+  g->T = T;
+  g->max_len = max_len;
+  g->total_blocks = blocks;
+  g->max_nc = (max_len - 1) / 4;
+  g->ld = std::max<int64_t>(4, round_up(std::max(g->max_nc, 1), 4));
+  g->score_tiles = static_cast<int32_t>(st);
+  g->attn_tiles = static_cast<int32_t>(at);
+  g->pl = make_plan_layout(g->R, g->topk);
+  g->max_words = (max_len - 1) / 4 / 32 + 1;
+  Carver c;
+  g->o_meta = c.take(sizeof(SeqMeta) * (num_seqs + 1));
+  g->o_kbar = c.take(static_cast<size_t>(std::max<int64_t>(blocks, 1)) * 64 * 2);
+  g->o_nc = c.take(static_cast<size_t>(T) * 4);
+  const int64_t rows = std::min<int64_t>(T, g->chunk_rows + 16);
+  g->o_scores = c.take(static_cast<size_t>(rows) * g->ld * 4);
+  g->o_idx = c.take(static_cast<size_t>(T) * g->topk * 4);
+  g->o_cnt = c.take(static_cast<size_t>(T) * 4);
+  g->o_plan = c.take(static_cast<size_t>(g->attn_tiles) * g->pl.stride * 4);
+  g->total = c.off;
+  return QSA_OK;
+}
+
+#define QSA_CHECK_LAUNCH()                                  \
+  do {                                                      \
+    cudaError_t e_ = cudaGetLastError();                    \
+    if (e_ != cudaSuccess) {                                \
+      fprintf(stderr, "qsa: launch failed: %s (%s:%d)\n",  \
+              cudaGetErrorString(e_), __FILE__, __LINE__);  \
+      return QSA_ERR_CUDA;                                  \
+    }                                                       \
+  } while (0)
+
+template <typename K>
+bool set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
+         cudaSuccess;
+}
+
+DevStatus dev_status(void* ws) { return DevStatus{reinterpret_cast<uint32_t*>(ws)}; }
+
+// ---- launch helpers ----------------------------------------------------------------
+qsa_status launch_meta(const int32_t* d_cu, int num_seqs, int R, SeqMeta* meta, DevStatus st,
+                       cudaStream_t s) {
+  k_seq_meta<<<1, 1024, 0, s>>>(d_cu, num_seqs, R, meta, st);
+  QSA_CHECK_LAUNCH();
+  return QSA_OK;
+}
+
+qsa_status launch_compress(const void* k_idx, const SeqMeta* meta, int num_seqs,
+                           int64_t total_blocks, void* kbar, cudaStream_t s) {
+  if (total_blocks == 0) return QSA_OK;
+  const int64_t n = total_blocks * 8;
+  const int threads = 256;
+  const int64_t want = (n + threads - 1) / threads;
+  const int grid = static_cast<int>(std::min<int64_t>(want, int64_t(num_sms()) * 16));
+  k_compress<<<grid, threads, 0, s>>>(reinterpret_cast<const uint4*>(k_idx), meta, num_seqs,
+                                      reinterpret_cast<uint4*>(kbar));
+  QSA_CHECK_LAUNCH();
+  return QSA_OK;
+}
+
+qsa_status launch_topk(const float* scores, int64_t ld, const int32_t* n_c, int64_t rows,
+                       int topk, int max_nc, int32_t* idx, int32_t* cnt, cudaStream_t s) {
+  if (rows <= 0) return QSA_OK;
+  const int cap = std::min(max_nc, kTopkSmemCap);
+  const int smem = 2048 * 4 + 64 * 4 + std::max(cap, 0) * 4;
+  if (!set_smem(k_topk, smem)) return QSA_ERR_CUDA;
+  const int grid = static_cast<int>(std::min<int64_t>(rows, int64_t(num_sms()) * 8));
+  k_topk<<<grid, kTopkThreads, smem, s>>>(scores, ld, n_c, rows, topk, cap, idx, cnt);
+  QSA_CHECK_LAUNCH();
+  return QSA_OK;
+}
+
+// Host-side token start of every 16-token score tile boundary, to cut score chunks.
+void score_tile_token_starts(const int32_t* h_cu, int num_seqs, std::vector<int64_t>* starts) {
+  starts->clear();
+  for (int s = 0; s < num_seqs; ++s) {
+    const int64_t L = h_cu[s + 1] - h_cu[s];
+    for (int64_t p = 0; p < L; p += 16) starts->push_back(h_cu[s] + p);
+  }
+  starts->push_back(h_cu[num_seqs]);
+}
+
+qsa_status run_scores_and_topk(const void* q_idx, const void* w, const void* kbar,
+                               const int32_t* h_cu, int num_seqs, const PrefillGeom& g,
+                               unsigned char* ws, int32_t* idx, int32_t* cnt, cudaStream_t s) {
+  SeqMeta* meta = reinterpret_cast<SeqMeta*>(ws + g.o_meta);
+  float* scores = reinterpret_cast<float*>(ws + g.o_scores);
+  const int32_t* n_c = reinterpret_cast<const int32_t*>(ws + g.o_nc);
+  CUtensorMap tm_kbar, tm_qidx;
+  {
+    const uint64_t dims[2] = {64, static_cast<uint64_t>(std::max<int64_t>(g.total_blocks, 1))};
+    const uint64_t strides[1] = {128};
+    const uint32_t box[2] = {64, 128};
+    if (!make_tmap(&tm_kbar, kbar, 2, dims, strides, box)) return QSA_ERR_CUDA;
+  }
+  {
+    const uint64_t dims[2] = {64, static_cast<uint64_t>(g.T) * 16};
+    const uint64_t strides[1] = {128};
+    const uint32_t box[2] = {64, 256};
+    if (!make_tmap(&tm_qidx, q_idx, 2, dims, strides, box)) return QSA_ERR_CUDA;
+  }
+  using C = ScoreCfg<16>;
+  const int smem = std::max(C::kSmemBytes, 116 * 1024);   // one CTA per SM (512 TMEM columns)
+  if (!set_smem(k_index_score<16>, smem)) return QSA_ERR_CUDA;
+  std::vector<int64_t> starts;
+  score_tile_token_starts(h_cu, num_seqs, &starts);
+  const int ntiles = static_cast<int>(starts.size()) - 1;
+  int t = 0;
+  while (t < ntiles) {
+    int e = t + 1;
+    while (e < ntiles && starts[e + 1] - starts[t] <= g.chunk_rows) ++e;
+    ScoreArgs a{};
+    a.meta = meta;
+    a.num_seqs = num_seqs;
+    a.tile_begin = t;
+    a.tile_count = e - t;
+    a.topk_skip = g.topk;
+    a.row_begin = starts[t];
+    a.w = reinterpret_cast<const __nv_bfloat16*>(w);
+    a.scores = scores;
+    a.ld = g.ld;
+    a.st = dev_status(ws);
+    k_index_score<16><<<e - t, C::kThreads, smem, s>>>(tm_kbar, tm_qidx, a);
+    QSA_CHECK_LAUNCH();
+    const int64_t r0 = starts[t], r1 = starts[e];
+    qsa_status st = launch_topk(scores, g.ld, n_c + r0, r1 - r0, g.topk, g.max_nc,
+                                idx + r0 * g.topk, cnt + r0, s);
+    if (st != QSA_OK) return st;
+    t = e;
+  }
+  return QSA_OK;
+}
+
+qsa_status run_attention(const void* q, const void* k, const void* v, const int32_t* idx,
+                         const int32_t* cnt, int num_seqs, const PrefillGeom& g,
+                         unsigned char* ws, void* out, cudaStream_t s) {
+  SeqMeta* meta = reinterpret_cast<SeqMeta*>(ws + g.o_meta);
+  int32_t* plan = reinterpret_cast<int32_t*>(ws + g.o_plan);
+  // union plans
+  {
+    const int mwords = g.pl.umax / 32;
+    const int smem = (2 * g.max_words + g.R * mwords) * 4;
+    if (!set_smem(k_attn_plan<false>, smem)) return QSA_ERR_CUDA;
+    const int grid = std::min(g.attn_tiles, num_sms() * 8);
+    k_attn_plan<false><<<grid, kPlanThreads, smem, s>>>(idx, cnt, g.topk, meta, num_seqs, nullptr,
+                                                        g.attn_tiles, g.pl, g.max_words, plan,
+                                                        dev_status(ws));
+    QSA_CHECK_LAUNCH();
+  }
+  CUtensorMap tm_q, tm_k, tm_v;
+  {
+    const uint64_t dims[3] = {128, 24, static_cast<uint64_t>(g.T)};
+    const uint64_t strides[2] = {256, 24 * 256};
+    const uint32_t box[3] = {64, 12, static_cast<uint32_t>(g.R)};
+    if (!make_tmap(&tm_q, q, 3, dims, strides, box)) return QSA_ERR_CUDA;
+  }
+  {
+    const uint64_t dims[2] = {256, static_cast<uint64_t>(g.T)};
+    const uint64_t strides[1] = {512};
+    const uint32_t box[2] = {64, 4};
+    if (!make_tmap(&tm_k, k, 2, dims, strides, box)) return QSA_ERR_CUDA;
+    if (!make_tmap(&tm_v, v, 2, dims, strides, box)) return QSA_ERR_CUDA;
+  }
+  if (!set_smem(k_sparse_attn, AttnCfg::kSmemBytes)) return QSA_ERR_CUDA;
+  AttnArgs a{};
+  a.plan = plan;
+  a.pl = g.pl;
+  a.meta = meta;
+  a.num_seqs = num_seqs;
+  a.decode = 0;
+  a.splits = 1;
+  a.out = reinterpret_cast<__nv_bfloat16*>(out);
+  a.st = dev_status(ws);
+  dim3 grid(g.attn_tiles, 2, 1);
+  k_sparse_attn<<<grid, AttnCfg::kThreads, AttnCfg::kSmemBytes, s>>>(tm_q, tm_k, tm_v, a);
+  QSA_CHECK_LAUNCH();
+  return QSA_OK;
+}
+
+qsa_status check_prefill_ptrs(std::initializer_list<const void*> ptrs) {
+  for (const void* p : ptrs) {
+    if (!p) return QSA_ERR_INVALID_ARG;
+    if (!aligned16(p)) return QSA_ERR_ALIGNMENT;
+  }
+  return QSA_OK;
+}
+
+// ---- decode geometry --------------------------------------------------------------------
+struct DecodeGeom {
+  int32_t B = 0, cap = 0, topk = 512, max_nc = 0, splits = 4;
+  int64_t ld = 4;
+  PlanLayout pl;
+  size_t o_scores = 0, o_nc = 0, o_idx = 0, o_cnt = 0, o_plan = 0, o_po = 0, o_pm = 0, o_pl = 0,
+         total = 0;
+};
+
+qsa_status decode_geom(const qsa_cache* c, const qsa_params& p, DecodeGeom* g) {
+  if (!c) return QSA_ERR_INVALID_ARG;
+  if (c->batch <= 0 || c->capacity <= 0 || c->capacity % 4 != 0 ||
+      c->capacity > QSA_MAX_SEQ_LEN)
+    return QSA_ERR_INVALID_ARG;
+  if (p.topk_blocks < 1 || p.topk_blocks > QSA_MAX_TOPK) return QSA_ERR_INVALID_ARG;
+  g->B = c->batch;
+  g->cap = c->capacity;
+  g->topk = p.topk_blocks;
+  g->max_nc = (c->capacity - 1) / 4;
+  g->ld = std::max<int64_t>(4, round_up(std::max(g->max_nc, 1), 4));
+  g->splits = p.decode_splits > 0 ? p.decode_splits : 4;
+  if (g->splits > 64) return QSA_ERR_INVALID_ARG;
+  g->pl = make_plan_layout(1, g->topk);
+  Carver cv;
+  g->o_scores = cv.take(static_cast<size_t>(g->B) * g->ld * 4);
+  g->o_nc = cv.take(static_cast<size_t>(g->B) * 4);
+  g->o_idx = cv.take(static_cast<size_t>(g->B) * g->topk * 4);
+  g->o_cnt = cv.take(static_cast<size_t>(g->B) * 4);
+  g->o_plan = cv.take(static_cast<size_t>(g->B) * g->pl.stride * 4);
+  const size_t parts = static_cast<size_t>(g->B) * 2 * g->splits * kGroup;
+  g->o_po = cv.take(parts * kHeadDim * 4);
+  g->o_pm = cv.take(parts * 4);
+  g->o_pl = cv.take(parts * 4);
+  g->total = cv.off;
+  return QSA_OK;
+}
+
+}  // namespace
+
+// =====================================================================================
+extern "C" {
+
+const char* qsa_status_string(qsa_status s) {
+  switch (s) {
+    case QSA_OK: return "QSA_OK";
+    case QSA_ERR_INVALID_ARG: return "QSA_ERR_INVALID_ARG";
+    case QSA_ERR_ALIGNMENT: return "QSA_ERR_ALIGNMENT";
+    case QSA_ERR_CAPACITY: return "QSA_ERR_CAPACITY";
+    case QSA_ERR_WORKSPACE: return "QSA_ERR_WORKSPACE";
+    case QSA_ERR_CUDA: return "QSA_ERR_CUDA";
+    case QSA_ERR_TIMEOUT: return "QSA_ERR_TIMEOUT";
+    case QSA_ERR_DEVICE: return "QSA_ERR_DEVICE";
+    case QSA_ERR_UNSUPPORTED: return "QSA_ERR_UNSUPPORTED";
+  }
+  return "QSA_ERR_UNKNOWN";
+}
+
+int32_t qsa_version(void) { return kVersion; }
+
+qsa_status qsa_workspace_init(void* workspace, size_t ws_bytes, qsa_stream_t stream) {
+  if (!workspace) return QSA_ERR_INVALID_ARG;
+  if (ws_bytes < QSA_WS_HEADER_BYTES) return QSA_ERR_WORKSPACE;
+  if (cudaMemsetAsync(workspace, 0, QSA_WS_HEADER_BYTES, reinterpret_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return QSA_ERR_CUDA;
+  return QSA_OK;
+}
+
+qsa_status qsa_last_device_error(void* workspace, qsa_stream_t stream, uint32_t* site) {
+  if (!workspace) return QSA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t h[4] = {0, 0, 0, 0};
+  if (cudaMemcpyAsync(h, workspace, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return QSA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return QSA_ERR_CUDA;
+  if (h[0] != 0) {
+    if (cudaMemsetAsync(workspace, 0, 16, s) != cudaSuccess) return QSA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return QSA_ERR_CUDA;
+  }
+  if (site) *site = h[1];
+  if (h[0] == 0) return QSA_OK;
+  return h[0] == kErrTimeout ? QSA_ERR_TIMEOUT : QSA_ERR_DEVICE;
+}
+
+// ---- step a1 -------------------------------------------------------------------------
+size_t qsa_compress_workspace_size(int32_t num_seqs) {
+  if (num_seqs <= 0) return 0;
+  Carver c;
+  c.take(sizeof(SeqMeta) * (num_seqs + 1));
+  return c.off;
+}
+
+qsa_status qsa_compress(const void* k_idx, const int32_t* d_cu_seqlens, const int32_t* h_cu_seqlens,
+                        int32_t num_seqs, void* kbar, void* workspace, size_t ws_bytes,
+                        qsa_stream_t stream) {
+  qsa_status st = check_prefill_ptrs({k_idx, d_cu_seqlens, kbar, workspace});
+  if (st != QSA_OK) return st;
+  qsa_params p{512, 1, 0, 0};
+  PrefillGeom g;
+  st = prefill_geom(h_cu_seqlens, num_seqs, p, &g);
+  if (st != QSA_OK) return st;
+  if (ws_bytes < qsa_compress_workspace_size(num_seqs)) return QSA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned char* ws = reinterpret_cast<unsigned char*>(workspace);
+  SeqMeta* meta = reinterpret_cast<SeqMeta*>(ws + QSA_WS_HEADER_BYTES);
+  st = launch_meta(d_cu_seqlens, num_seqs, 1, meta, dev_status(ws), s);
+  if (st != QSA_OK) return st;
+  return launch_compress(k_idx, meta, num_seqs, g.total_blocks, kbar, s);
+}
+
+// ---- step a2 alone -----------------------------------------------------------------------
+qsa_status qsa_index_scores(const void* q_idx, const void* w, const void* kbar,
+                            const int32_t* d_cu_seqlens, const int32_t* h_cu_seqlens,
+                            int32_t num_seqs, int64_t row_begin, int64_t row_end, float* scores,
+                            int64_t ld, int32_t topk, void* workspace, size_t ws_bytes,
+                            qsa_stream_t stream) {
+  qsa_status st = check_prefill_ptrs({q_idx, w, kbar, d_cu_seqlens, scores, workspace});
+  if (st != QSA_OK) return st;
+  qsa_params p{topk > 0 ? topk : 512, 1, 0, 0};
+  PrefillGeom g;
+  st = prefill_geom(h_cu_seqlens, num_seqs, p, &g);
+  if (st != QSA_OK) return st;
+  if (ws_bytes < g.total) return QSA_ERR_WORKSPACE;
+  if (ld < std::max<int64_t>(g.max_nc, 1) || ld % 4 != 0) return QSA_ERR_INVALID_ARG;
+  if (row_begin < 0 || row_end > g.T || row_begin >= row_end) return QSA_ERR_INVALID_ARG;
+  std::vector<int64_t> starts;
+  score_tile_token_starts(h_cu_seqlens, num_seqs, &starts);
+  const auto tb = std::lower_bound(starts.begin(), starts.end(), row_begin);
+  const auto te = std::lower_bound(starts.begin(), starts.end(), row_end);
+  if (tb == starts.end() || *tb != row_begin || te == starts.end() || *te != row_end)
+    return QSA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned char* ws = reinterpret_cast<unsigned char*>(workspace);
+  SeqMeta* meta = reinterpret_cast<SeqMeta*>(ws + g.o_meta);
+  st = launch_meta(d_cu_seqlens, num_seqs, g.R, meta, dev_status(ws), s);
+  if (st != QSA_OK) return st;
+  CUtensorMap tm_kbar, tm_qidx;
+  {
+    const uint64_t dims[2] = {64, static_cast<uint64_t>(std::max<int64_t>(g.total_blocks, 1))};
+    const uint64_t strides[1] = {128};
+    const uint32_t box[2] = {64, 128};
+    if (!make_tmap(&tm_kbar, kbar, 2, dims, strides, box)) return QSA_ERR_CUDA;
+  }
+  {
+    const uint64_t dims[2] = {64, static_cast<uint64_t>(g.T) * 16};
+    const uint64_t strides[1] = {128};
+    const uint32_t box[2] = {64, 256};
+    if (!make_tmap(&tm_qidx, q_idx, 2, dims, strides, box)) return QSA_ERR_CUDA;
+  }
+  using C = ScoreCfg<16>;
+  const int smem = std::max(C::kSmemBytes, 116 * 1024);
+  if (!set_smem(k_index_score<16>, smem)) return QSA_ERR_CUDA;
+  ScoreArgs a{};
+  a.meta = meta;
+  a.num_seqs = num_seqs;
+  a.tile_begin = static_cast<int32_t>(tb - starts.begin());
+  a.tile_count = static_cast<int32_t>(te - tb);
+  a.topk_skip = topk > 0 ? topk : 0;
+  a.row_begin = row_begin;
+  a.w = reinterpret_cast<const __nv_bfloat16*>(w);
+  a.scores = scores;
+  a.ld = ld;
+  a.st = dev_status(ws);
+  k_index_score<16><<<a.tile_count, C::kThreads, smem, s>>>(tm_kbar, tm_qidx, a);
+  QSA_CHECK_LAUNCH();
+  return QSA_OK;
+}
+
+// ---- step a3 alone -----------------------------------------------------------------------
+qsa_status qsa_topk(const float* scores, int64_t ld, const int32_t* n_c, int64_t rows, int32_t topk,
+                    int32_t max_n_c, int32_t* idx, int32_t* cnt, qsa_stream_t stream) {
+  qsa_status st = check_prefill_ptrs({scores, n_c, idx, cnt});
+  if (st != QSA_OK) return st;
+  if (rows <= 0 || topk < 1 || topk > QSA_MAX_TOPK || max_n_c < 0 || ld < std::max(max_n_c, 1))
+    return QSA_ERR_INVALID_ARG;
+  return launch_topk(scores, ld, n_c, rows, topk, max_n_c, idx, cnt,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+// ---- prefill -----------------------------------------------------------------------------
+size_t qsa_prefill_workspace_size(const int32_t* h_cu_seqlens, int32_t num_seqs, qsa_params params) {
+  PrefillGeom g;
+  if (prefill_geom(h_cu_seqlens, num_seqs, params, &g) != QSA_OK) return 0;
+  return g.total;
+}
+
+static qsa_status prefill_common(const void* q, const void* k, const void* v, const void* q_idx,
+                                 const void* k_idx, const void* w, const int32_t* d_cu,
+                                 const int32_t* h_cu, int32_t num_seqs, void* out, int32_t* idx_ext,
+                                 int32_t* cnt_ext, const int32_t* idx_in, const int32_t* cnt_in,
+                                 void* workspace, size_t ws_bytes, qsa_params params,
+                                 qsa_stream_t stream) {
+  PrefillGeom g;
+  qsa_status st = prefill_geom(h_cu, num_seqs, params, &g);
+  if (st != QSA_OK) return st;
+  if (ws_bytes < g.total) return QSA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned char* ws = reinterpret_cast<unsigned char*>(workspace);
+  SeqMeta* meta = reinterpret_cast<SeqMeta*>(ws + g.o_meta);
+  st = launch_meta(d_cu, num_seqs, g.R, meta, dev_status(ws), s);
+  if (st != QSA_OK) return st;
+  const int32_t* idx_use = idx_in;
+  const int32_t* cnt_use = cnt_in;
+  if (!idx_in) {
+    int32_t* idx = idx_ext ? idx_ext : reinterpret_cast<int32_t*>(ws + g.o_idx);
+    int32_t* cnt = cnt_ext ? cnt_ext : reinterpret_cast<int32_t*>(ws + g.o_cnt);
+    void* kbar = ws + g.o_kbar;
+    st = launch_compress(k_idx, meta, num_seqs, g.total_blocks, kbar, s);
+    if (st != QSA_OK) return st;
+    {
+      const int64_t threads = 256;
+      const int grid = static_cast<int>(std::min<int64_t>((g.T + threads - 1) / threads,
+                                                          int64_t(num_sms()) * 8));
+      k_row_nc<<<grid, threads, 0, s>>>(meta, num_seqs, g.T, reinterpret_cast<int32_t*>(ws + g.o_nc));
+      QSA_CHECK_LAUNCH();
+    }
+    st = run_scores_and_topk(q_idx, w, kbar, h_cu, num_seqs, g, ws, idx, cnt, s);
+    if (st != QSA_OK) return st;
+    idx_use = idx;
+    cnt_use = cnt;
+  }
+  if (out) return run_attention(q, k, v, idx_use, cnt_use, num_seqs, g, ws, out, s);
+  return QSA_OK;
+}
+
+qsa_status qsa_prefill(const void* q, const void* k, const void* v, const void* q_idx,
+                       const void* k_idx, const void* w, const int32_t* d_cu_seqlens,
+                       const int32_t* h_cu_seqlens, int32_t num_seqs, void* out, void* workspace,
+                       size_t ws_bytes, qsa_params params, qsa_stream_t stream) {
+  qsa_status st = check_prefill_ptrs({q, k, v, q_idx, k_idx, w, d_cu_seqlens, out, workspace});
+  if (st != QSA_OK) return st;
+  return prefill_common(q, k, v, q_idx, k_idx, w, d_cu_seqlens, h_cu_seqlens, num_seqs, out,
+                        nullptr, nullptr, nullptr, nullptr, workspace, ws_bytes, params, stream);
+}
+
+qsa_status qsa_prefill_select(const void* q_idx, const void* k_idx, const void* w,
+                              const int32_t* d_cu_seqlens, const int32_t* h_cu_seqlens,
+                              int32_t num_seqs, int32_t* idx, int32_t* cnt, void* workspace,
+                              size_t ws_bytes, qsa_params params, qsa_stream_t stream) {
+  qsa_status st = check_prefill_ptrs({q_idx, k_idx, w, d_cu_seqlens, idx, cnt, workspace});
+  if (st != QSA_OK) return st;
+  return prefill_common(nullptr, nullptr, nullptr, q_idx, k_idx, w, d_cu_seqlens, h_cu_seqlens,
+                        num_seqs, nullptr, idx, cnt, nullptr, nullptr, workspace, ws_bytes, params,
+                        stream);
+}
+
+qsa_status qsa_sparse_attention(const void* q, const void* k, const void* v, const int32_t* idx,
+                                const int32_t* cnt, const int32_t* d_cu_seqlens,
+                                const int32_t* h_cu_seqlens, int32_t num_seqs, void* out,
+                                void* workspace, size_t ws_bytes, qsa_params params,
+                                qsa_stream_t stream) {
+  qsa_status st = check_prefill_ptrs({q, k, v, idx, cnt, d_cu_seqlens, out, workspace});
+  if (st != QSA_OK) return st;
+  return prefill_common(q, k, v, nullptr, nullptr, nullptr, d_cu_seqlens, h_cu_seqlens, num_seqs,
+                        out, nullptr, nullptr, idx, cnt, workspace, ws_bytes, params, stream);
+}
+
+// ---- append ------------------------------------------------------------------------------
+qsa_status qsa_append_kv(const qsa_cache* cache, const void* k, const void* v, const void* k_idx,
+                         int32_t n_new, const int32_t* counts, const int32_t* h_len,
+                         qsa_stream_t stream) {
+  if (!cache || !h_len) return QSA_ERR_INVALID_ARG;
+  qsa_status st = check_prefill_ptrs({k, v, k_idx, cache->k_blocks, cache->v_blocks, cache->kbar,
+                                      cache->kbar_partial, cache->len});
+  if (st != QSA_OK) return st;
+  if (counts && !aligned16(counts)) return QSA_ERR_ALIGNMENT;
+  if (cache->batch <= 0 || cache->capacity <= 0 || cache->capacity % 4 != 0 ||
+      cache->capacity > QSA_MAX_SEQ_LEN || n_new < 0)
+    return QSA_ERR_INVALID_ARG;
+  if (n_new == 0) return QSA_OK;
+  for (int b = 0; b < cache->batch; ++b) {
+    if (h_len[b] < 0 || h_len[b] > cache->capacity) return QSA_ERR_INVALID_ARG;
+    if (!counts && static_cast<int64_t>(h_len[b]) + n_new > cache->capacity) return QSA_ERR_CAPACITY;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  AppendParams p{};
+  p.k = reinterpret_cast<const uint4*>(k);
+  p.v = reinterpret_cast<const uint4*>(v);
+  p.k_idx = reinterpret_cast<const uint4*>(k_idx);
+  p.counts = counts;
+  p.n_new = n_new;
+  p.batch = cache->batch;
+  p.capacity = cache->capacity;
+  p.k_blocks = reinterpret_cast<uint4*>(cache->k_blocks);
+  p.v_blocks = reinterpret_cast<uint4*>(cache->v_blocks);
+  p.kbar = reinterpret_cast<uint4*>(cache->kbar);
+  p.partial = cache->kbar_partial;
+  p.len = cache->len;
+  p.st = DevStatus{nullptr};
+  const int sms = num_sms();
+  {
+    const int64_t n = static_cast<int64_t>(p.batch) * n_new * 32;
+    const int grid = static_cast<int>(std::min<int64_t>((n + 255) / 256, int64_t(sms) * 16));
+    k_append_kv_copy<<<grid, 256, 0, s>>>(p);
+    QSA_CHECK_LAUNCH();
+  }
+  {
+    const int slots = (n_new + 3) / 4 + 1;
+    const int64_t n = static_cast<int64_t>(p.batch) * slots * 8;
+    const int grid = static_cast<int>(std::min<int64_t>((n + 255) / 256, int64_t(sms) * 16));
+    k_append_kbar<<<grid, 256, 0, s>>>(p, slots);
+    QSA_CHECK_LAUNCH();
+  }
+  k_append_len<<<(p.batch + 255) / 256, 256, 0, s>>>(cache->len, counts, n_new, p.batch);
+  QSA_CHECK_LAUNCH();
+  return QSA_OK;
+}
+
+// ---- decode --------------------------------------------------------------------------------
+size_t qsa_decode_workspace_size(const qsa_cache* cache, qsa_params params) {
+  DecodeGeom g;
+  if (decode_geom(cache, params, &g) != QSA_OK) return 0;
+  return g.total;
+}
+
+qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, const void* w,
+                      void* out, const int32_t* h_len, int32_t* sel_idx, int32_t* sel_cnt,
+                      void* workspace, size_t ws_bytes, qsa_params params, qsa_stream_t stream) {
+  if (!cache || !h_len) return QSA_ERR_INVALID_ARG;
+  qsa_status st = check_prefill_ptrs({q, q_idx, w, out, workspace, cache->k_blocks,
+                                      cache->v_blocks, cache->kbar, cache->len});
+  if (st != QSA_OK) return st;
+  if ((sel_idx && !aligned16(sel_idx)) || (sel_cnt && !aligned16(sel_cnt))) return QSA_ERR_ALIGNMENT;
+  DecodeGeom g;
+  st = decode_geom(cache, params, &g);
+  if (st != QSA_OK) return st;
+  if (ws_bytes < g.total) return QSA_ERR_WORKSPACE;
+  int max_len = 0;
+  for (int b = 0; b < g.B; ++b) {
+    if (h_len[b] < 1 || h_len[b] > g.cap) return QSA_ERR_INVALID_ARG;
+    max_len = std::max(max_len, h_len[b]);
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned char* ws = reinterpret_cast<unsigned char*>(workspace);
+  float* scores = reinterpret_cast<float*>(ws + g.o_scores);
+  int32_t* n_c = reinterpret_cast<int32_t*>(ws + g.o_nc);
+  int32_t* idx = sel_idx ? sel_idx : reinterpret_cast<int32_t*>(ws + g.o_idx);
+  int32_t* cnt = sel_cnt ? sel_cnt : reinterpret_cast<int32_t*>(ws + g.o_cnt);
+  int32_t* plan = reinterpret_cast<int32_t*>(ws + g.o_plan);
+  const int sms = num_sms();
+  const int max_nc_now = (max_len - 1) / 4;
+  // a2: scores (one token x 16 heads per sequence, split over M-tiles)
+  {
+    CUtensorMap tm_kbar, tm_qidx;
+    const uint64_t dk[2] = {64, static_cast<uint64_t>(g.B) * (g.cap / 4)};
+    const uint64_t sk[1] = {128};
+    const uint32_t bk[2] = {64, 128};
+    if (!make_tmap(&tm_kbar, cache->kbar, 2, dk, sk, bk)) return QSA_ERR_CUDA;
+    const uint64_t dq[2] = {64, static_cast<uint64_t>(g.B) * 16};
+    const uint32_t bq[2] = {64, 16};
+    if (!make_tmap(&tm_qidx, q_idx, 2, dq, sk, bq)) return QSA_ERR_CUDA;
+    using C = ScoreCfg<1>;
+    if (!set_smem(k_index_score<1>, C::kSmemBytes)) return QSA_ERR_CUDA;
+    const int total_mt = std::max(1, (max_nc_now + 127) / 128);
+    int splits = std::max(1, (2 * sms + g.B - 1) / g.B);
+    splits = std::min(splits, total_mt);
+    const int per = (total_mt + splits - 1) / splits;
+    splits = (total_mt + per - 1) / per;
+    ScoreArgs a{};
+    a.len = cache->len;
+    a.splits = splits;
+    a.mtiles_per_split = per;
+    a.kbar_rows_per_seq = g.cap / 4;
+    a.n_c_out = n_c;
+    a.w = reinterpret_cast<const __nv_bfloat16*>(w);
+    a.scores = scores;
+    a.ld = g.ld;
+    a.st = dev_status(ws);
+    k_index_score<1><<<g.B * splits, C::kThreads, C::kSmemBytes, s>>>(tm_kbar, tm_qidx, a);
+    QSA_CHECK_LAUNCH();
+  }
+  // a3: top-k
+  st = launch_topk(scores, g.ld, n_c, g.B, g.topk, max_nc_now, idx, cnt, s);
+  if (st != QSA_OK) return st;
+  // union plan (one token per tile)
+  {
+    const int max_words = (g.cap - 1) / 4 / 32 + 1;
+    const int mwords = g.pl.umax / 32;
+    const int smem = (2 * max_words + mwords) * 4;
+    if (!set_smem(k_attn_plan<true>, smem)) return QSA_ERR_CUDA;
+    k_attn_plan<true><<<std::min(g.B, sms * 8), kPlanThreads, smem, s>>>(
+        idx, cnt, g.topk, nullptr, 0, cache->len, g.B, g.pl, max_words, plan, dev_status(ws));
+    QSA_CHECK_LAUNCH();
+  }
+  // a6: split attention + combine
+  {
+    CUtensorMap tm_q, tm_k, tm_v;
+    const uint64_t dq[3] = {128, 24, static_cast<uint64_t>(g.B)};
+    const uint64_t sq[2] = {256, 24 * 256};
+    const uint32_t bq[3] = {64, 12, 1};
+    if (!make_tmap(&tm_q, q, 3, dq, sq, bq)) return QSA_ERR_CUDA;
+    const uint64_t dkv[2] = {128, static_cast<uint64_t>(g.B) * 2 * g.cap};
+    const uint64_t skv[1] = {256};
+    const uint32_t bkv[2] = {64, 4};
+    if (!make_tmap(&tm_k, cache->k_blocks, 2, dkv, skv, bkv)) return QSA_ERR_CUDA;
+    if (!make_tmap(&tm_v, cache->v_blocks, 2, dkv, skv, bkv)) return QSA_ERR_CUDA;
+    if (!set_smem(k_sparse_attn, AttnCfg::kSmemBytes)) return QSA_ERR_CUDA;
+    AttnArgs a{};
+    a.plan = plan;
+    a.pl = g.pl;
+    a.decode = 1;
+    a.splits = g.splits;
+    a.cap_blocks = g.cap / 4;
+    a.part_o = reinterpret_cast<float*>(ws + g.o_po);
+    a.part_m = reinterpret_cast<float*>(ws + g.o_pm);
+    a.part_l = reinterpret_cast<float*>(ws + g.o_pl);
+    a.st = dev_status(ws);
+    dim3 grid(g.B, 2, g.splits);
+    k_sparse_attn<<<grid, AttnCfg::kThreads, AttnCfg::kSmemBytes, s>>>(tm_q, tm_k, tm_v, a);
+    QSA_CHECK_LAUNCH();
+    const int warps = g.B * kHeads;
+    k_decode_combine<<<(warps * 32 + 255) / 256, 256, 0, s>>>(a.part_o, a.part_m, a.part_l, g.B,
+                                                              g.splits,
+                                                              reinterpret_cast<__nv_bfloat16*>(out));
+    QSA_CHECK_LAUNCH();
+  }
+  return QSA_OK;
+}
+
+}  // extern "C"

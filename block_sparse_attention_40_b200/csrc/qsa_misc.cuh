@@ -1,0 +1,623 @@
+// qsa_misc.cuh -- bandwidth-bound QSA kernels: sequence metadata, block compression,
+// cache append, radix top-k, the attention union plan and the decode split combine.
+#pragma once
+
+#include "qsa_common.cuh"
+
+namespace qsa {
+
+// Per-sequence metadata derived on the device from cu_seqlens.
+struct SeqMeta {
+  int64_t tok0;      // first token of the sequence in the packed arrays
+  int64_t kbar0;     // first compressed block of the sequence in the packed kbar array
+  int32_t len;       // tokens
+  int32_t score_tile0;  // first 16-token score tile (global numbering)
+  int32_t attn_tile0;   // first attention tile (rows_per_tile tokens each)
+  int32_t pad;
+};
+
+// ---------------------------------------------------------------------------------------
+// Block-wide exclusive scan of one int per thread (blockDim.x a multiple of 32, <= 1024).
+__device__ __forceinline__ int block_excl_scan(int v, int* sh /*[33]*/, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nw = (blockDim.x + 31) >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sh[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int y = lane < nw ? sh[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int z = __shfl_up_sync(0xffffffffu, y, o);
+      if (lane >= o) y += z;
+    }
+    sh[lane] = y;   // inclusive prefix of warp totals
+  }
+  __syncthreads();
+  int excl = x - v + (warp > 0 ? sh[warp - 1] : 0);
+  *total = sh[nw - 1];
+  __syncthreads();
+  return excl;
+}
+
+// One CTA: metadata for every sequence (prefix sums over blocks and tiles).
+__global__ void __launch_bounds__(1024) k_seq_meta(const int32_t* __restrict__ cu, int num_seqs,
+                                                   int rows_per_tile, SeqMeta* __restrict__ meta,
+                                                   DevStatus st) {
+  __shared__ int sh[33];
+  int64_t carry_blk = 0;
+  int carry_st = 0, carry_at = 0;
+  for (int base = 0; base < num_seqs; base += blockDim.x) {
+    const int s = base + threadIdx.x;
+    int L = 0;
+    int64_t t0 = 0;
+    if (s < num_seqs) {
+      t0 = cu[s];
+      L = cu[s + 1] - cu[s];
+      if (L < 0) {
+        report_error(st, kErrDevice, 100);
+        L = 0;
+      }
+    }
+    const int nb = L / kBlock, nst = (L + 15) / 16,
+              nat = rows_per_tile > 0 ? (L + rows_per_tile - 1) / rows_per_tile : 0;
+    int tot_b, tot_s, tot_a;
+    const int eb = block_excl_scan(nb, sh, &tot_b);
+    const int es = block_excl_scan(nst, sh, &tot_s);
+    const int ea = block_excl_scan(nat, sh, &tot_a);
+    if (s < num_seqs) {
+      SeqMeta m;
+      m.tok0 = t0;
+      m.kbar0 = carry_blk + eb;
+      m.len = L;
+      m.score_tile0 = carry_st + es;
+      m.attn_tile0 = carry_at + ea;
+      m.pad = 0;
+      meta[s] = m;
+    }
+    carry_blk += tot_b;
+    carry_st += tot_s;
+    carry_at += tot_a;
+  }
+  if (threadIdx.x == 0) {   // sentinel entry: totals
+    SeqMeta m;
+    m.tok0 = 0;
+    m.kbar0 = carry_blk;
+    m.len = 0;
+    m.score_tile0 = carry_st;
+    m.attn_tile0 = carry_at;
+    m.pad = 0;
+    meta[num_seqs] = m;
+  }
+}
+
+// Sequence owning global tile `gt` (tile0 of meta is non-decreasing; meta[num_seqs] holds totals).
+template <bool kAttnTiles>
+__device__ __forceinline__ int find_seq_of_tile(const SeqMeta* meta, int num_seqs, int gt) {
+  int lo = 0, hi = num_seqs - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    const int t0 = kAttnTiles ? meta[mid].attn_tile0 : meta[mid].score_tile0;
+    if (t0 <= gt) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ int find_seq_of_token(const SeqMeta* meta, int num_seqs, int64_t t) {
+  int lo = 0, hi = num_seqs - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (meta[mid].tok0 <= t) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// n_c (number of candidate blocks) of every token row: floor(pos / 4).
+__global__ void k_row_nc(const SeqMeta* __restrict__ meta, int num_seqs, int64_t total,
+                         int32_t* __restrict__ n_c) {
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total;
+       t += (int64_t)gridDim.x * blockDim.x) {
+    const int s = find_seq_of_token(meta, num_seqs, t);
+    n_c[t] = static_cast<int32_t>((t - meta[s].tok0) / kBlock);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Step a1, fixed order: kbar = bf16_rne(((k0 + k1) + k2) + k3) * 0.25) with fp32 sums.
+// One thread per (block, 8-dim slice): four 16-byte loads, one 16-byte store.
+__device__ __forceinline__ uint4 compress4(uint4 a, uint4 b, uint4 c, uint4 d) {
+  const uint32_t* pa = reinterpret_cast<const uint32_t*>(&a);
+  const uint32_t* pb = reinterpret_cast<const uint32_t*>(&b);
+  const uint32_t* pc = reinterpret_cast<const uint32_t*>(&c);
+  const uint32_t* pd = reinterpret_cast<const uint32_t*>(&d);
+  uint4 out;
+  uint32_t* po = reinterpret_cast<uint32_t*>(&out);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float lo = __uint_as_float(pa[i] << 16), hi = __uint_as_float(pa[i] & 0xffff0000u);
+    lo = __fadd_rn(lo, __uint_as_float(pb[i] << 16));
+    hi = __fadd_rn(hi, __uint_as_float(pb[i] & 0xffff0000u));
+    lo = __fadd_rn(lo, __uint_as_float(pc[i] << 16));
+    hi = __fadd_rn(hi, __uint_as_float(pc[i] & 0xffff0000u));
+    lo = __fadd_rn(lo, __uint_as_float(pd[i] << 16));
+    hi = __fadd_rn(hi, __uint_as_float(pd[i] & 0xffff0000u));
+    po[i] = pack_bf16x2(__fmul_rn(lo, 0.25f), __fmul_rn(hi, 0.25f));
+  }
+  return out;
+}
+
+__global__ void k_compress(const uint4* __restrict__ k_idx, const SeqMeta* __restrict__ meta,
+                           int num_seqs, uint4* __restrict__ kbar) {
+  const int64_t total_blocks = meta[num_seqs].kbar0;
+  const int64_t n = total_blocks * 8;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t gb = i >> 3;
+    const int part = static_cast<int>(i & 7);
+    // sequence of packed block gb: last s with kbar0 <= gb
+    int lo = 0, hi = num_seqs - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (meta[mid].kbar0 <= gb) lo = mid; else hi = mid - 1;
+    }
+    const int64_t b = gb - meta[lo].kbar0;
+    const int64_t tok = meta[lo].tok0 + 4 * b;
+    const uint4* src = k_idx + tok * 8 + part;
+    kbar[gb * 8 + part] = compress4(src[0], src[8], src[16], src[24]);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Step a5: append.  Part 1 copies K/V rows into the blocked cache and (re)computes the
+// compressed keys of the blocks the new tokens touch.  The first touched block may hold
+// older tokens whose running sum is in kbar_partial; the last touched block may stay
+// incomplete and leaves its sum there.  The same thread handles both ends of a sequence
+// so that the read of the old partial precedes the write of the new one.
+struct AppendParams {
+  const uint4* k;      // [B][n_new][2][128] bf16 as 16-byte units
+  const uint4* v;
+  const uint4* k_idx;  // [B][n_new][64]
+  const int32_t* counts;  // [B] or null
+  int32_t n_new;
+  int32_t batch;
+  int32_t capacity;
+  uint4* k_blocks;     // [B][2][cap/4][4][128]
+  uint4* v_blocks;
+  uint4* kbar;         // [B][cap/4][64]
+  float* partial;      // [B][64]
+  const int32_t* len;  // [B]
+  DevStatus st;
+};
+
+__device__ __forceinline__ int append_count(const AppendParams& p, int b) {
+  int c = p.counts ? p.counts[b] : p.n_new;
+  return c < 0 ? 0 : (c > p.n_new ? p.n_new : c);
+}
+
+// Copies: one thread per 16 bytes of K or V.
+__global__ void k_append_kv_copy(AppendParams p) {
+  const int64_t per_tok = 2 * 16;                       // 2 heads x 16 units of 16 B
+  const int64_t n = static_cast<int64_t>(p.batch) * p.n_new * per_tok;
+  const int64_t cap_blk = p.capacity / kBlock;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int b = static_cast<int>(i / (static_cast<int64_t>(p.n_new) * per_tok));
+    const int64_t rem = i - static_cast<int64_t>(b) * p.n_new * per_tok;
+    const int j = static_cast<int>(rem / per_tok);
+    const int g = static_cast<int>((rem / 16) & 1);
+    const int u = static_cast<int>(rem & 15);
+    if (j >= append_count(p, b)) continue;
+    const int64_t pos = static_cast<int64_t>(p.len[b]) + j;
+    if (pos >= p.capacity) {
+      report_error(p.st, kErrDevice, 200);
+      continue;
+    }
+    const int64_t dst = ((((static_cast<int64_t>(b) * 2 + g) * cap_blk + pos / 4) * 4 + pos % 4) *
+                         16) + u;
+    const int64_t src = ((static_cast<int64_t>(b) * p.n_new + j) * 2 + g) * 16 + u;
+    p.k_blocks[dst] = p.k[src];
+    p.v_blocks[dst] = p.v[src];
+    // The last appended token of a sequence zeroes the rest of its block, so that rows not
+    // yet written are finite (attention reads whole blocks and masks the future rows).
+    if (j == append_count(p, b) - 1) {
+      for (int64_t q = pos + 1; q < (pos / 4) * 4 + 4; ++q) {
+        const int64_t dz = ((((static_cast<int64_t>(b) * 2 + g) * cap_blk + q / 4) * 4 + q % 4) *
+                            16) + u;
+        p.k_blocks[dz] = make_uint4(0, 0, 0, 0);
+        p.v_blocks[dz] = make_uint4(0, 0, 0, 0);
+      }
+    }
+  }
+}
+
+// Compressed keys: one thread per (sequence, touched block, 8-dim slice).  Slot 0 of each
+// sequence handles the first and the last touched block; slots 1.. the complete middle ones.
+__global__ void k_append_kbar(AppendParams p, int max_blocks_touched) {
+  const int64_t slots = static_cast<int64_t>(max_blocks_touched);
+  const int64_t n = static_cast<int64_t>(p.batch) * slots * 8;
+  const int64_t cap_blk = p.capacity / kBlock;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int b = static_cast<int>(i / (slots * 8));
+    const int64_t slot = (i / 8) % slots;
+    const int part = static_cast<int>(i & 7);
+    const int cnt = append_count(p, b);
+    if (cnt == 0) continue;
+    const int64_t L0 = p.len[b];
+    const int64_t L1 = L0 + cnt;
+    if (L1 > p.capacity) {
+      if (slot == 0 && part == 0) report_error(p.st, kErrDevice, 201);
+      continue;
+    }
+    const int64_t jf = L0 / 4, jl = (L1 - 1) / 4;
+    const uint4* kin = p.k_idx + static_cast<int64_t>(b) * p.n_new * 8 + part;  // token j at +8j
+    float* part_sum = p.partial + static_cast<int64_t>(b) * 64 + part * 8;
+    uint4* kb_out = p.kbar + (static_cast<int64_t>(b) * cap_blk) * 8 + part;
+    auto add_tokens = [&](float* acc, int64_t from, int64_t to, bool start_from_first) {
+      // sum tokens [from, to) (absolute positions) into acc in order
+      for (int64_t pos = from; pos < to; ++pos) {
+        const uint4 x = kin[(pos - L0) * 8];
+        const uint32_t* px = reinterpret_cast<const uint32_t*>(&x);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float lo = __uint_as_float(px[q] << 16), hi = __uint_as_float(px[q] & 0xffff0000u);
+          if (start_from_first && pos == from) {
+            acc[2 * q] = lo;
+            acc[2 * q + 1] = hi;
+          } else {
+            acc[2 * q] = __fadd_rn(acc[2 * q], lo);
+            acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], hi);
+          }
+        }
+      }
+    };
+    auto finish = [&](const float* acc, int64_t j, bool complete) {
+      if (complete) {
+        uint4 o;
+        uint32_t* po = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          po[q] = pack_bf16x2(__fmul_rn(acc[2 * q], 0.25f), __fmul_rn(acc[2 * q + 1], 0.25f));
+        kb_out[j * 8] = o;
+      } else {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) part_sum[q] = acc[q];
+      }
+    };
+    float acc[8];
+    if (slot == 0) {
+      // first touched block
+      const int64_t end_f = (4 * jf + 4 < L1) ? 4 * jf + 4 : L1;
+      if (L0 % 4 != 0) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] = part_sum[q];
+        add_tokens(acc, L0, end_f, false);
+      } else {
+        add_tokens(acc, L0, end_f, true);
+      }
+      finish(acc, jf, end_f == 4 * jf + 4);
+      if (jl != jf) {   // last touched block starts fresh
+        add_tokens(acc, 4 * jl, L1, true);
+        finish(acc, jl, L1 == 4 * jl + 4);
+      }
+    } else {
+      const int64_t j = jf + slot;       // middle blocks jf+1 .. jl-1 are complete and new
+      if (j >= jl) continue;
+      add_tokens(acc, 4 * j, 4 * j + 4, true);
+      finish(acc, j, true);
+    }
+  }
+}
+
+__global__ void k_append_len(int32_t* len, const int32_t* counts, int32_t n_new, int batch) {
+  for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < batch; b += gridDim.x * blockDim.x) {
+    int c = counts ? counts[b] : n_new;
+    c = c < 0 ? 0 : (c > n_new ? n_new : c);
+    len[b] += c;
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Step a3: top-k per row by radix select on order-preserving uint32 keys (11+11+10 bits),
+// then an ordered compaction that emits the selected blocks in ascending index order and
+// breaks ties at the threshold toward lower indices.  One 512-thread CTA per row.
+constexpr int kTopkThreads = 512;
+
+__device__ __forceinline__ float topk_load(const float* src, int i) { return src[i]; }
+
+__global__ void __launch_bounds__(kTopkThreads) k_topk(const float* __restrict__ scores,
+                                                       int64_t ld, const int32_t* __restrict__ n_c,
+                                                       int64_t rows, int topk, int smem_cap,
+                                                       int32_t* __restrict__ idx,
+                                                       int32_t* __restrict__ cnt) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw);          // 2048
+  int* sh = reinterpret_cast<int*>(hist + 2048);                     // 33 (+ pad)
+  int* sel = sh + 40;                                                // 2
+  float* row_cache = reinterpret_cast<float*>(smem_raw + 2048 * 4 + 64 * 4);
+  const int tid = threadIdx.x;
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const int n = n_c[r];
+    int32_t* out = idx + r * topk;
+    if (n <= topk) {
+      for (int i = tid; i < topk; i += blockDim.x) out[i] = i < n ? i : -1;
+      if (tid == 0) cnt[r] = n < 0 ? 0 : n;
+      continue;
+    }
+    const float* src = scores + r * ld;
+    if (n <= smem_cap) {
+      for (int i = tid; i < n; i += blockDim.x) row_cache[i] = src[i];
+      src = row_cache;
+      __syncthreads();
+    }
+    uint32_t prefix = 0, pmask = 0;
+    int need = topk;
+    const int shifts[3] = {21, 10, 0};
+    const int bitsv[3] = {11, 11, 10};
+    for (int pass = 0; pass < 3; ++pass) {
+      const int shift = shifts[pass];
+      const int nbins = 1 << bitsv[pass];
+      const uint32_t bmask = static_cast<uint32_t>(nbins - 1);
+      for (int i = tid; i < 2048; i += blockDim.x) hist[i] = 0;
+      __syncthreads();
+      for (int i = tid; i < n; i += blockDim.x) {
+        const uint32_t key = float_key(src[i]);
+        if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & bmask], 1u);
+      }
+      __syncthreads();
+      // suffix scan over bins (from the highest bin down)
+      const int per = nbins / kTopkThreads;   // 4 or 2
+      const int rt = kTopkThreads - 1 - tid;  // thread owning the highest bins has rt = 0
+      const int b_hi = (tid + 1) * per - 1;   // my highest bin
+      int local = 0;
+      for (int q = 0; q < per; ++q) local += static_cast<int>(hist[b_hi - q]);
+      int tot;
+      // exclusive scan in rt order == sum over threads with higher tid
+      // (threads are reordered through the rt index)
+      __shared__ int sh_rt[kTopkThreads];
+      sh_rt[rt] = local;
+      __syncthreads();
+      const int v = sh_rt[tid];   // value of the thread whose rt == tid
+      const int ex = block_excl_scan(v, sh, &tot);
+      sh_rt[tid] = ex;            // exclusive prefix for rt == tid
+      __syncthreads();
+      int running = sh_rt[rt];
+      for (int q = 0; q < per; ++q) {
+        const int bin = b_hi - q;
+        const int h = static_cast<int>(hist[bin]);
+        if (running < need && running + h >= need) {
+          sel[0] = bin;
+          sel[1] = running;
+        }
+        running += h;
+      }
+      __syncthreads();
+      const int bin = sel[0];
+      need -= sel[1];
+      prefix |= static_cast<uint32_t>(bin) << shift;
+      pmask |= bmask << shift;
+      __syncthreads();
+    }
+    const uint32_t T = prefix;
+    const int need_eq = need;   // elements equal to T to take (lowest indices first)
+    int base_out = 0, eq_seen = 0;
+    for (int start = 0; start < n; start += blockDim.x) {
+      const int i = start + tid;
+      uint32_t key = 0;
+      if (i < n) key = float_key(src[i]);
+      const int gt = (i < n && key > T) ? 1 : 0;
+      const int eq = (i < n && key == T) ? 1 : 0;
+      int eq_tot;
+      const int eq_rank = eq_seen + block_excl_scan(eq, sh, &eq_tot);
+      const int take = (gt || (eq && eq_rank < need_eq)) ? 1 : 0;
+      int take_tot;
+      const int pos = base_out + block_excl_scan(take, sh, &take_tot);
+      if (take && pos < topk) out[pos] = i;
+      base_out += take_tot;
+      eq_seen += eq_tot;
+      if (base_out >= topk) break;
+    }
+    if (tid == 0) cnt[r] = topk;
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Attention plan.  A tile is up to R consecutive query tokens of one sequence (R = 1 for
+// decode).  The tile's key set is the union U of its tokens' selected blocks and their own
+// blocks, in ascending block order.  For every token r and every 32-block chunk q of the
+// union, mask[r][q] has bit u set when union block 32q+u is selected by r or is r's own
+// block; tail[r] is the union position of r's own block.
+struct PlanLayout {
+  int32_t R;         // tokens per tile
+  int32_t umax;      // union capacity per tile (multiple of 32)
+  int64_t stride;    // int32 entries per tile record
+  // record: [0] = U, [1] = number of tokens, [2..2+R) = tail positions,
+  //         [2+R .. 2+R+umax) = union block ids, then R * (umax/32) mask words
+  __host__ __device__ int64_t union_off() const { return 2 + R; }
+  __host__ __device__ int64_t mask_off() const { return 2 + R + umax; }
+};
+
+__host__ __device__ inline PlanLayout make_plan_layout(int R, int topk) {
+  PlanLayout pl;
+  pl.R = R;
+  pl.umax = ((R * (topk + 1)) + 31) / 32 * 32;
+  pl.stride = 2 + R + pl.umax + static_cast<int64_t>(R) * (pl.umax / 32);
+  pl.stride = (pl.stride + 3) / 4 * 4;   // 16-byte aligned records
+  return pl;
+}
+
+constexpr int kPlanThreads = 256;
+
+// kDecode: tile = sequence b, single token at p = len[b]-1, selection rows idx[b].
+template <bool kDecode>
+__global__ void __launch_bounds__(kPlanThreads) k_attn_plan(
+    const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt, int topk,
+    const SeqMeta* __restrict__ meta, int num_seqs, const int32_t* __restrict__ len,
+    int num_tiles, PlanLayout pl, int max_words, int32_t* __restrict__ plan, DevStatus st) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  uint32_t* bitmap = reinterpret_cast<uint32_t*>(smem_raw);          // max_words
+  int* wpref = reinterpret_cast<int*>(bitmap + max_words);            // max_words
+  uint32_t* masks = reinterpret_cast<uint32_t*>(wpref + max_words);   // R * umax/32
+  __shared__ int sh[33];
+  __shared__ int64_t s_row0;
+  __shared__ int s_pos0, s_ntok;
+  const int tid = threadIdx.x;
+  const int mwords = pl.umax / 32;
+  for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    if (tid == 0) {
+      if (kDecode) {
+        s_row0 = tile;
+        s_pos0 = len[tile] - 1;
+        s_ntok = 1;
+      } else {
+        const int s = find_seq_of_tile<true>(meta, num_seqs, tile);
+        const int lt = tile - meta[s].attn_tile0;
+        const int p0 = lt * pl.R;
+        s_pos0 = p0;
+        s_row0 = meta[s].tok0 + p0;
+        const int rem = meta[s].len - p0;
+        s_ntok = rem < pl.R ? rem : pl.R;
+      }
+    }
+    __syncthreads();
+    const int ntok = s_ntok, pos0 = s_pos0;
+    const int64_t row0 = s_row0;
+    int32_t* rec = plan + static_cast<int64_t>(tile) * pl.stride;
+    if (ntok <= 0 || pos0 < 0) {
+      if (tid == 0) {
+        rec[0] = 0;
+        rec[1] = 0;
+      }
+      __syncthreads();
+      continue;
+    }
+    const int c_last = (pos0 + ntok - 1) / kBlock;
+    const int nwords = c_last / 32 + 1;
+    if (nwords > max_words) {
+      if (tid == 0) {
+        report_error(st, kErrDevice, 300);
+        rec[0] = 0;
+        rec[1] = 0;
+      }
+      __syncthreads();
+      continue;
+    }
+    for (int i = tid; i < nwords; i += blockDim.x) bitmap[i] = 0;
+    for (int i = tid; i < pl.R * mwords; i += blockDim.x) masks[i] = 0;
+    __syncthreads();
+    // mark selected blocks and own blocks
+    for (int r = 0; r < ntok; ++r) {
+      const int c_r = (pos0 + r) / kBlock;
+      const int n = cnt[row0 + r];
+      const int32_t* ir = idx + (row0 + r) * topk;
+      for (int j = tid; j < n; j += blockDim.x) {
+        const int b = ir[j];
+        if (b < 0 || b >= c_r) {
+          report_error(st, kErrDevice, 301);
+          continue;
+        }
+        atomicOr(&bitmap[b >> 5], 1u << (b & 31));
+      }
+      if (tid == 0) atomicOr(&bitmap[c_r >> 5], 1u << (c_r & 31));
+    }
+    __syncthreads();
+    // prefix popcounts over bitmap words
+    int carry = 0;
+    for (int base = 0; base < nwords; base += blockDim.x) {
+      const int w = base + tid;
+      const int pc = w < nwords ? __popc(bitmap[w]) : 0;
+      int tot;
+      const int ex = block_excl_scan(pc, sh, &tot);
+      if (w < nwords) wpref[w] = carry + ex;
+      carry += tot;
+    }
+    __syncthreads();
+    const int U = carry;
+    if (U > pl.umax) {   // cannot happen for valid selections
+      if (tid == 0) {
+        report_error(st, kErrDevice, 302);
+        rec[0] = 0;
+        rec[1] = 0;
+      }
+      __syncthreads();
+      continue;
+    }
+    int32_t* uni = rec + pl.union_off();
+    for (int w = tid; w < nwords; w += blockDim.x) {
+      uint32_t bits = bitmap[w];
+      int pos = wpref[w];
+      while (bits) {
+        const int bit = __ffs(bits) - 1;
+        bits &= bits - 1;
+        uni[pos++] = w * 32 + bit;
+      }
+    }
+    // masks and tails
+    for (int r = 0; r < ntok; ++r) {
+      const int c_r = (pos0 + r) / kBlock;
+      const int n = cnt[row0 + r];
+      const int32_t* ir = idx + (row0 + r) * topk;
+      for (int j = tid; j <= n; j += blockDim.x) {
+        int b = (j < n) ? ir[j] : c_r;
+        if (b < 0 || b > c_r) continue;
+        const int w = b >> 5;
+        const int pos = wpref[w] + __popc(bitmap[w] & ((1u << (b & 31)) - 1u));
+        atomicOr(&masks[r * mwords + (pos >> 5)], 1u << (pos & 31));
+        if (j == n) rec[2 + r] = pos;
+      }
+    }
+    __syncthreads();
+    const int nq = (U + 31) / 32;
+    uint32_t* mout = reinterpret_cast<uint32_t*>(rec + pl.mask_off());
+    for (int i = tid; i < ntok * mwords; i += blockDim.x) {
+      const int r = i / mwords, q = i % mwords;
+      if (q < nq) mout[r * mwords + q] = masks[r * mwords + q];
+    }
+    if (tid == 0) {
+      rec[0] = U;
+      rec[1] = ntok;
+    }
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Decode: merge the split partials of each (sequence, head) by log-sum-exp.
+//   partial O (unnormalised, fp32) [B][2][splits][12][128]; m (log2 domain), l [B][2][splits][12]
+__global__ void k_decode_combine(const float* __restrict__ part_o, const float* __restrict__ part_m,
+                                 const float* __restrict__ part_l, int batch, int splits,
+                                 __nv_bfloat16* __restrict__ out) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= batch * kHeads) return;
+  const int b = warp / kHeads, h = warp % kHeads, g = h / kGroup, hr = h % kGroup;
+  const int64_t base = (static_cast<int64_t>(b) * 2 + g) * splits;
+  float M = -INFINITY;
+  for (int s = 0; s < splits; ++s) M = fmaxf(M, part_m[(base + s) * kGroup + hr]);
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  float L = 0.f;
+  for (int s = 0; s < splits; ++s) {
+    const float m = part_m[(base + s) * kGroup + hr];
+    const float f = (m == -INFINITY) ? 0.f : exp2f(m - M);
+    L += f * part_l[(base + s) * kGroup + hr];
+    const float4 o = reinterpret_cast<const float4*>(
+        part_o + ((base + s) * kGroup + hr) * kHeadDim)[lane];
+    acc[0] += f * o.x;
+    acc[1] += f * o.y;
+    acc[2] += f * o.z;
+    acc[3] += f * o.w;
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  uint2 pk;
+  pk.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  pk.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+  reinterpret_cast<uint2*>(out + (static_cast<int64_t>(b) * kHeads + h) * kHeadDim)[lane] = pk;
+}
+
+}  // namespace qsa

@@ -1,0 +1,268 @@
+// qsa_score.cuh -- step a2, the MQA indexer score, on tcgen05 tensor cores.
+//
+//   s(t, b) = sum_h w[t,h] * ReLU(q_idx[t,h] . kbar[b])      (16 heads, width 64)
+//
+// A dense contraction: D[block, (token, head)] = kbar[block, :] . q_idx[(token, head), :]
+// with M = 128 compressed blocks per tile (A operand, streamed by TMA), N = 16 tokens x 16
+// heads = 256 (prefill) or 1 token x 16 heads (decode) (B operand, loaded once per CTA),
+// K = 64.  The fp32 accumulator lives in TMEM (two buffers, so the epilogue of tile i
+// overlaps the MMA of tile i+1).  Epilogue: each thread owns one block row, reads its
+// 16 heads per token from TMEM, applies ReLU, weights by w and sums in fp32, and writes
+// the score if the block is a candidate of that token (b < floor(pos/4)).
+//
+// Warp roles: warp 0 issues TMA, warp 1 allocates TMEM and issues MMAs (one thread),
+// the remaining warps run the epilogue.
+#pragma once
+
+#include "qsa_common.cuh"
+#include "qsa_misc.cuh"
+
+namespace qsa {
+
+template <int NTOK>
+struct ScoreCfg {
+  static constexpr int kN = NTOK * kIdxHeads;             // MMA N
+  static constexpr int kAccCols = kN < 32 ? 32 : kN;      // TMEM columns per accumulator
+  static constexpr int kNumAcc = NTOK == 16 ? 2 : 4;
+  static constexpr int kTmemCols = kAccCols * kNumAcc;    // 512 / 128
+  static constexpr int kStages = NTOK == 16 ? 4 : 8;
+  static constexpr int kEpiWarps = NTOK == 16 ? 8 : 4;
+  static constexpr int kThreads = 64 + 32 * kEpiWarps;
+  static constexpr int kABytes = 128 * kIdxDim * 2;       // 16 KB
+  static constexpr int kBBytes = kN * kIdxDim * 2;        // 32 KB / 2 KB
+  static constexpr int kBOff = kStages * kABytes;
+  static constexpr int kWOff = kBOff + ((kBBytes + 1023) / 1024) * 1024;
+  static constexpr int kBarOff = kWOff + NTOK * kIdxHeads * 4;
+  static constexpr int kNumBars = 2 * kStages + 2 * kNumAcc + 2;
+  static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;  // + align slack
+  static constexpr uint32_t kIdesc = idesc_bf16_f32(128, kN, 0, 0);
+};
+
+struct ScoreArgs {
+  // prefill
+  const SeqMeta* meta;
+  int32_t num_seqs;
+  int32_t tile_begin;      // global 16-token tile range [tile_begin, tile_begin + gridDim.x)
+  int32_t tile_count;
+  int32_t topk_skip;       // skip tiles whose largest n_c <= topk_skip (0 = none)
+  int64_t row_begin;       // score row 0 corresponds to this global token
+  // decode
+  const int32_t* len;      // [B]
+  int32_t splits;
+  int32_t mtiles_per_split;
+  int64_t kbar_rows_per_seq;
+  int32_t* n_c_out;        // [B] n_c per sequence (written by split 0), may be null
+  // common
+  const __nv_bfloat16* w;  // prefill: [T][16]; decode: [B][16]
+  float* scores;
+  int64_t ld;
+  DevStatus st;
+};
+
+template <int NTOK>
+struct ScoreWork {
+  int64_t a_row0;    // first kbar row of this CTA's first M-tile
+  int32_t mt0;       // first M-tile index (block offset = 128 * (mt0 + i))
+  int32_t n_mtiles;
+  int32_t b_row0;    // first q_idx row (token * 16)
+  int32_t ntok;      // valid tokens in the N tile
+  int32_t pos0;      // position (within the sequence) of token 0
+  int64_t out_row0;  // score row of token 0
+};
+
+template <int NTOK>
+__device__ __forceinline__ ScoreWork<NTOK> score_work(const ScoreArgs& a) {
+  ScoreWork<NTOK> wk;
+  if constexpr (NTOK == 16) {
+    const int gt = a.tile_begin + (a.tile_count - 1 - static_cast<int>(blockIdx.x));
+    const int s = find_seq_of_tile<false>(a.meta, a.num_seqs, gt);
+    const SeqMeta m = a.meta[s];
+    const int lt = gt - m.score_tile0;
+    const int p0 = lt * 16;
+    const int ntok = (m.len - p0) < 16 ? (m.len - p0) : 16;
+    const int c_max = (p0 + ntok - 1) / kBlock;
+    wk.ntok = ntok;
+    wk.pos0 = p0;
+    wk.mt0 = 0;
+    wk.n_mtiles = (ntok <= 0 || c_max <= a.topk_skip) ? 0 : (c_max + 127) / 128;
+    wk.a_row0 = m.kbar0;
+    wk.b_row0 = static_cast<int32_t>((m.tok0 + p0) * kIdxHeads);
+    wk.out_row0 = m.tok0 + p0 - a.row_begin;
+  } else {
+    const int b = static_cast<int>(blockIdx.x) / a.splits;
+    const int split = static_cast<int>(blockIdx.x) % a.splits;
+    const int p = a.len[b] - 1;
+    const int n_c = p >= 0 ? p / kBlock : 0;
+    if (split == 0 && threadIdx.x == 0 && a.n_c_out) a.n_c_out[b] = n_c;
+    const int total = (n_c + 127) / 128;
+    const int m0 = split * a.mtiles_per_split;
+    int m1 = m0 + a.mtiles_per_split;
+    if (m1 > total) m1 = total;
+    wk.ntok = 1;
+    wk.pos0 = p;
+    wk.mt0 = m0;
+    wk.n_mtiles = m1 > m0 ? m1 - m0 : 0;
+    wk.a_row0 = static_cast<int64_t>(b) * a.kbar_rows_per_seq;
+    wk.b_row0 = b * kIdxHeads;
+    wk.out_row0 = b;
+  }
+  return wk;
+}
+
+template <int NTOK>
+__global__ void __launch_bounds__(ScoreCfg<NTOK>::kThreads, 1)
+    k_index_score(const __grid_constant__ CUtensorMap tmap_kbar,
+                  const __grid_constant__ CUtensorMap tmap_qidx, ScoreArgs args) {
+  using C = ScoreCfg<NTOK>;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  unsigned char* sA = smem;
+  unsigned char* sB = smem + C::kBOff;
+  float* sW = reinterpret_cast<float*>(smem + C::kWOff);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + C::kStages;
+  uint64_t* acc_full = bars + 2 * C::kStages;
+  uint64_t* acc_empty = acc_full + C::kNumAcc;
+  uint64_t* b_full = acc_empty + C::kNumAcc;
+  uint64_t* mma_done = b_full + 1;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+
+  const ScoreWork<NTOK> wk = score_work<NTOK>(args);
+  if (wk.n_mtiles <= 0) return;   // uniform over the CTA
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < C::kNumAcc; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], C::kEpiWarps);
+    }
+    mbar_init(b_full, 1);
+    mbar_init(mma_done, 1);
+    *s_abort = 0;
+    fence_mbar_init();
+  }
+  // weights of the tile's tokens, widened to fp32
+  for (int i = threadIdx.x; i < NTOK * kIdxHeads; i += blockDim.x) {
+    const int tok = i / kIdxHeads;
+    float wv = 0.f;
+    if (tok < wk.ntok) {
+      const int64_t row = static_cast<int64_t>(wk.b_row0) + i;   // b_row0 = token*16
+      wv = __bfloat162float(args.w[row]);
+    }
+    sW[i] = wv;
+  }
+  if (warp == 1) {
+    tmem_alloc(s_tmem, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      prefetch_tmap(&tmap_kbar);
+      prefetch_tmap(&tmap_qidx);
+      mbar_arrive_expect_tx(b_full, C::kBBytes);
+      tma_load_2d(sB, &tmap_qidx, 0, wk.b_row0, b_full);
+      int issued = 0;
+      for (int i = 0; i < wk.n_mtiles; ++i) {
+        const int s = i % C::kStages;
+        if (!mbar_wait(&empty[s], ((i / C::kStages) & 1) ^ 1, s_abort, args.st, 10)) break;
+        mbar_arrive_expect_tx(&full[s], C::kABytes);
+        tma_load_2d(sA + s * C::kABytes, &tmap_kbar, 0,
+                    static_cast<int32_t>(wk.a_row0 + 128ll * (wk.mt0 + i)), &full[s]);
+        ++issued;
+      }
+      if (*s_abort) {
+        // let copies already in flight land before the CTA exits
+        const int from = issued > C::kStages ? issued - C::kStages : 0;
+        for (int j = from; j < issued; ++j) mbar_drain(&full[j % C::kStages], (j / C::kStages) & 1);
+        mbar_drain(b_full, 0);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      bool ok = mbar_wait(b_full, 0, s_abort, args.st, 11);
+      const uint32_t sA0 = smem_u32(sA), sB0 = smem_u32(sB);
+      for (int i = 0; ok && i < wk.n_mtiles; ++i) {
+        const int s = i % C::kStages;
+        const int a = i % C::kNumAcc;
+        if (!mbar_wait(&full[s], (i / C::kStages) & 1, s_abort, args.st, 12)) break;
+        if (!mbar_wait(&acc_empty[a], ((i / C::kNumAcc) & 1) ^ 1, s_abort, args.st, 13)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + a * C::kAccCols;
+#pragma unroll
+        for (int k = 0; k < kIdxDim / 16; ++k) {
+          const uint64_t da = smem_desc_sw128(sA0 + s * C::kABytes + 32 * k, 0, 1024);
+          const uint64_t db = smem_desc_sw128(sB0 + 32 * k, 0, 1024);
+          umma_ss(d, da, db, C::kIdesc, k > 0 ? 1u : 0u);
+        }
+        umma_commit(&empty[s]);
+        umma_commit(&acc_full[a]);
+      }
+      umma_commit(mma_done);
+      mbar_drain(mma_done, 0);
+    }
+  } else {
+    // ---------------- epilogue ----------------
+    const int ew = warp - 2;
+    const int quarter = warp & 3;          // TMEM lanes this warp may access
+    const int part = ew / 4;               // which half of the tokens (prefill)
+    constexpr int kTokPerWarp = NTOK == 16 ? 8 : 1;
+    const int tok_base = part * kTokPerWarp;
+    for (int i = 0; i < wk.n_mtiles; ++i) {
+      const int a = i % C::kNumAcc;
+      const bool got = mbar_wait(&acc_full[a], (i / C::kNumAcc) & 1, s_abort, args.st, 14);
+      if (__any_sync(0xffffffffu, !got)) break;   // also reconverges the warp
+      tc_fence_after();
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + a * C::kAccCols +
+                             tok_base * kIdxHeads;
+      uint32_t acc[kTokPerWarp * kIdxHeads];
+      if constexpr (NTOK == 16) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tbase + 32 * c, acc + 32 * c);
+      } else {
+        tmem_ld16(tbase, acc);
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[a]);
+      const int blk = 128 * (wk.mt0 + i) + quarter * 32 + lane;
+#pragma unroll
+      for (int j = 0; j < kTokPerWarp; ++j) {
+        const int tok = tok_base + j;
+        float s = 0.f;
+#pragma unroll
+        for (int h = 0; h < kIdxHeads; ++h) {
+          const float x = __uint_as_float(acc[j * kIdxHeads + h]);
+          s = fmaf(sW[tok * kIdxHeads + h], fmaxf(x, 0.f), s);
+        }
+        const int pos = wk.pos0 + tok;
+        if (tok < wk.ntok && blk < pos / kBlock)
+          args.scores[(wk.out_row0 + tok) * args.ld + blk] = s;
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace qsa

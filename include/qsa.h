@@ -1,0 +1,229 @@
+/*
+ * qsa.h -- C ABI of the B200 (sm_100a) Qwen Sparse Attention library (libqsa.so).
+ *
+ * The method (sources on the pages):
+ *   - "Long context became an architecture problem", section "Linear attention carries
+ *     the stream; sparse attention retrieves detail": a small indexer scores compressed
+ *     key blocks and picks the relevant ones; the budget is 512 blocks (2,048 tokens);
+ *     the final incomplete block stays uncompressed.
+ *   - axbrief "unsloth Qwen3.8-Flash-Next GGUF", section "Shifting from Tokens to
+ *     Micro-Blocks": micro-block processing; 24 query heads paired with 2 KV heads.
+ *   - "Qwen3.8-Flash-Next Previews Qwen4.x Architecture", FAQ: 4-token micro-blocks.
+ *   - aiany.app "Qwen3.8-Flash-Next", "Key Capabilities": the indexer is MQA.
+ *   - aiany.app, "Implementation notes": KV cache sizing for very long contexts.
+ * Parameters the pages leave open, fixed here: head_dim 128; a block's compressed key is
+ * the fp32 mean of its 4 per-token indexer keys (summed in token order, stored as bf16
+ * round-to-nearest-even); 16 indexer query heads of width 64 sharing one key head; score
+ * s(t,b) = sum_h w[t,h] * ReLU(q_idx[t,h] . kbar[b]); one block selection per token for all
+ * 24 heads; top-k ties go to the lower block index.
+ *
+ * Per sequence, token t (0-based) may select among the complete blocks 0 .. floor(t/4)-1
+ * (strictly before its own block, even when its own block is complete), keeps the
+ * min(k, floor(t/4)) best, and attends to their 4k tokens plus its own block's tokens
+ * 4*floor(t/4) .. t, with one softmax (scale 1/sqrt(128)); query head h reads KV head h/12.
+ *
+ * Conventions for every call:
+ *   - All tensor arguments are DEVICE pointers, 16-byte aligned, contiguous, row-major in
+ *     the layouts stated, owned by the caller.  The library never allocates device memory;
+ *     scratch space is the caller's `workspace` (size from the *_workspace_size query).
+ *   - `h_*` arguments are HOST pointers read synchronously during the call.
+ *   - Work is enqueued on `stream` (NULL = the legacy default stream) and the call returns
+ *     without synchronising.  Host-detectable errors are returned before anything is
+ *     enqueued.  Device-side failures (a bounded wait that timed out, an index out of
+ *     range) are recorded in the first 16 bytes of the workspace and reported by
+ *     qsa_last_device_error().
+ *   - bf16 means IEEE bfloat16 (raw 16-bit); fp32 is IEEE single.
+ *   - Calls are re-entrant; the only global state is a per-device cache of driver entry
+ *     points.  Concurrent calls must not share a workspace.
+ */
+#ifndef QSA_H_
+#define QSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define QSA_API __attribute__((visibility("default")))
+#else
+#define QSA_API
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st *qsa_stream_t;   /* same object as a cudaStream_t */
+
+#define QSA_NUM_HEADS 24
+#define QSA_NUM_KV_HEADS 2
+#define QSA_HEAD_DIM 128
+#define QSA_IDX_HEADS 16
+#define QSA_IDX_DIM 64
+#define QSA_BLOCK 4
+#define QSA_MAX_TOPK 1024          /* largest supported budget k (the pages use 512) */
+#define QSA_MAX_SEQ_LEN 1048576    /* longest supported sequence / cache, in tokens */
+#define QSA_WS_HEADER_BYTES 256    /* status words at the start of every workspace */
+
+typedef enum {
+  QSA_OK = 0,
+  QSA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, bad lengths */
+  QSA_ERR_ALIGNMENT = 2,     /* a pointer is not 16-byte aligned */
+  QSA_ERR_CAPACITY = 3,      /* an append would exceed the cache capacity */
+  QSA_ERR_WORKSPACE = 4,     /* workspace too small */
+  QSA_ERR_CUDA = 5,          /* a CUDA runtime/driver call failed (launch, tensor map) */
+  QSA_ERR_TIMEOUT = 6,       /* device: a bounded wait gave up */
+  QSA_ERR_DEVICE = 7,        /* device: an out-of-range index was found and skipped */
+  QSA_ERR_UNSUPPORTED = 8    /* valid request outside this build's limits */
+} qsa_status;
+
+typedef struct {
+  int32_t topk_blocks;     /* budget k in blocks, 1..QSA_MAX_TOPK (512 on the pages) */
+  int32_t rows_per_tile;   /* prefill attention: query tokens packed into one 128-row
+                              tensor-core tile (1..10); 0 = library default */
+  int32_t decode_splits;   /* decode attention: key splits per (sequence, KV head);
+                              0 = library default */
+  int32_t score_chunk_rows;/* prefill: query rows scored per pass (bounds the score
+                              buffer in the workspace); 0 = library default */
+} qsa_params;
+
+/* KV cache for decode.  Blocks of 4 tokens are contiguous per (sequence, KV head):
+ *   k_blocks, v_blocks : bf16 [batch][2][capacity/4][4][128]   (1 KB per block)
+ *   kbar               : bf16 [batch][capacity/4][64]          compressed indexer keys
+ *   kbar_partial       : fp32 [batch][64]  running sum of the current incomplete block
+ *   len                : int32 [batch]     tokens stored per sequence (device)
+ * capacity is a multiple of 4, at most QSA_MAX_SEQ_LEN.  All buffers are caller-owned;
+ * zero-initialise len before the first append. */
+typedef struct {
+  void *k_blocks;
+  void *v_blocks;
+  void *kbar;
+  float *kbar_partial;
+  int32_t *len;
+  int32_t batch;
+  int32_t capacity;
+} qsa_cache;
+
+/* Human-readable name of a status code (static string). */
+QSA_API const char *qsa_status_string(qsa_status s);
+
+/* Library version (major*10000 + minor*100 + patch). */
+QSA_API int32_t qsa_version(void);
+
+/* Zero the status words at the start of a workspace (enqueued on stream).  Call once
+ * after allocating a workspace, before its first use. */
+QSA_API qsa_status qsa_workspace_init(void *workspace, size_t ws_bytes, qsa_stream_t stream);
+
+/* Synchronise `stream`, read and clear the device status word of `workspace`.  Returns
+ * QSA_OK, QSA_ERR_TIMEOUT or QSA_ERR_DEVICE (the first failure recorded since the last
+ * read), or QSA_ERR_CUDA if the synchronisation itself failed.  If site != NULL it receives
+ * an internal id of the failing wait / check. */
+QSA_API qsa_status qsa_last_device_error(void *workspace, qsa_stream_t stream, uint32_t *site);
+
+/* ---------------------------------------------------------------------------------- */
+/* Step a1: block compression ("Long context became an architecture problem": the indexer
+ * scores compressed key blocks; the mean is this library's choice of compression).
+ *   k_idx         bf16 [T][64]   per-token indexer keys, sequences packed back to back
+ *   d_cu_seqlens  int32 [num_seqs+1] device copy of the cumulative lengths (cu[0] = 0)
+ *   h_cu_seqlens  int32 [num_seqs+1] host copy of the same values
+ *   kbar          bf16 [sum_s floor(L_s/4)][64] output, sequence s starting at block
+ *                 sum_{j<s} floor(L_j/4)
+ * kbar[b][d] = bf16_rne(((k0 + k1) + k2) + k3) * 0.25) with fp32 sums; only complete
+ * blocks are written (a trailing partial block "remains uncompressed").  The workspace
+ * (qsa_compress_workspace_size bytes) holds per-sequence offsets. */
+QSA_API size_t qsa_compress_workspace_size(int32_t num_seqs);
+
+QSA_API qsa_status qsa_compress(const void *k_idx, const int32_t *d_cu_seqlens,
+                        const int32_t *h_cu_seqlens, int32_t num_seqs, void *kbar,
+                        void *workspace, size_t ws_bytes, qsa_stream_t stream);
+
+/* Step a2 alone (prefill shape): indexer scores of query rows [row_begin, row_end) against
+ * the compressed keys of their own sequence.  workspace: qsa_prefill_workspace_size bytes
+ * (only its header and per-sequence metadata are used).
+ *   q_idx   bf16 [T][16][64];  w bf16 [T][16];  kbar as written by qsa_compress
+ *   scores  fp32 [row_end-row_begin][ld]: scores[t-row_begin][b] = s(t,b) for every
+ *           b < floor(pos(t)/4); other entries are left untouched.  ld >= max n_c.
+ * row_begin/row_end must fall on 16-token tile boundaries of their sequences (a sequence
+ * start, a multiple of 16 tokens into a sequence, or the end of a sequence).
+ * Rows whose candidates all fit in topk (floor(pos/4) <= topk) may be skipped when
+ * topk > 0; pass topk = 0 to score every row. */
+QSA_API qsa_status qsa_index_scores(const void *q_idx, const void *w, const void *kbar,
+                            const int32_t *d_cu_seqlens, const int32_t *h_cu_seqlens,
+                            int32_t num_seqs, int64_t row_begin, int64_t row_end,
+                            float *scores, int64_t ld, int32_t topk, void *workspace,
+                            size_t ws_bytes, qsa_stream_t stream);
+
+/* Step a3 alone: per-row top-k ("Long context ...": budget 512 blocks = 2,048 tokens;
+ * ties to the lower block index).
+ *   scores  fp32 [rows][ld], row r has n_c[r] candidates in columns 0..n_c[r]-1
+ *   n_c     int32 [rows] (device)
+ *   idx     int32 [rows][topk] output: the min(topk, n_c) selected blocks in ascending
+ *           order, padded with -1;  cnt int32 [rows] output: min(topk, n_c). */
+QSA_API qsa_status qsa_topk(const float *scores, int64_t ld, const int32_t *n_c, int64_t rows,
+                    int32_t topk, int32_t max_n_c, int32_t *idx, int32_t *cnt,
+                    qsa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------- */
+/* Prefill (steps a1-a4) over a packed varlen batch.
+ *   q      bf16 [T][24][128]      k, v   bf16 [T][2][128]
+ *   q_idx  bf16 [T][16][64]       k_idx  bf16 [T][64]       w  bf16 [T][16] (w >= 0)
+ *   out    bf16 [T][24][128]
+ * Sequence lengths >= 1 and <= QSA_MAX_SEQ_LEN. */
+QSA_API size_t qsa_prefill_workspace_size(const int32_t *h_cu_seqlens, int32_t num_seqs,
+                                  qsa_params params);
+
+QSA_API qsa_status qsa_prefill(const void *q, const void *k, const void *v, const void *q_idx,
+                       const void *k_idx, const void *w, const int32_t *d_cu_seqlens,
+                       const int32_t *h_cu_seqlens, int32_t num_seqs, void *out,
+                       void *workspace, size_t ws_bytes, qsa_params params,
+                       qsa_stream_t stream);
+
+/* Steps a1-a3 only: the block selection of every token.
+ *   idx int32 [T][topk] (ascending, -1 padded),  cnt int32 [T]. */
+QSA_API qsa_status qsa_prefill_select(const void *q_idx, const void *k_idx, const void *w,
+                              const int32_t *d_cu_seqlens, const int32_t *h_cu_seqlens,
+                              int32_t num_seqs, int32_t *idx, int32_t *cnt, void *workspace,
+                              size_t ws_bytes, qsa_params params, qsa_stream_t stream);
+
+/* Step a4 alone: attention of every token over a given selection (idx/cnt as returned by
+ * qsa_prefill_select) plus its own block.  Selected blocks must be < floor(pos/4),
+ * ascending, without repeats. */
+QSA_API qsa_status qsa_sparse_attention(const void *q, const void *k, const void *v, const int32_t *idx,
+                                const int32_t *cnt, const int32_t *d_cu_seqlens,
+                                const int32_t *h_cu_seqlens, int32_t num_seqs, void *out,
+                                void *workspace, size_t ws_bytes, qsa_params params,
+                                qsa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------- */
+/* Step a5: append tokens to the cache (aiany.app "Implementation notes": KV cache sizing
+ * for very long contexts).  For each sequence b, counts[b] (or n_new if counts is NULL)
+ * tokens are appended after its current length:
+ *   k, v   bf16 [batch][n_new][2][128]     k_idx  bf16 [batch][n_new][64]
+ *   counts int32 [batch] device, each 0..n_new, or NULL
+ *   h_len  int32 [batch] HOST copy of the current lengths, used to check capacity.
+ * Complete blocks get their compressed key with exactly the bits qsa_compress would
+ * produce; an incomplete last block keeps its running fp32 sum in kbar_partial.
+ * len is advanced on the device. */
+QSA_API qsa_status qsa_append_kv(const qsa_cache *cache, const void *k, const void *v,
+                         const void *k_idx, int32_t n_new, const int32_t *counts,
+                         const int32_t *h_len, qsa_stream_t stream);
+
+/* Decode (steps a2, a3, a6) for one new query token per sequence, at position
+ * p = len-1 (its K/V/k_idx must already be appended).
+ *   q      bf16 [batch][24][128]    q_idx bf16 [batch][16][64]    w bf16 [batch][16]
+ *   out    bf16 [batch][24][128]
+ *   h_len  int32 [batch] HOST copy of the lengths after the append (sizes the grids).
+ * Optional outputs sel_idx int32 [batch][topk] / sel_cnt int32 [batch] receive the block
+ * selection (pass NULL to skip). */
+QSA_API size_t qsa_decode_workspace_size(const qsa_cache *cache, qsa_params params);
+
+QSA_API qsa_status qsa_decode(const void *q, const qsa_cache *cache, const void *q_idx, const void *w,
+                      void *out, const int32_t *h_len, int32_t *sel_idx, int32_t *sel_cnt,
+                      void *workspace, size_t ws_bytes, qsa_params params,
+                      qsa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QSA_H_ */

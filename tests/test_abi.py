@@ -1,0 +1,108 @@
+"""The C ABI library builds, loads and exports every entry point that include/qsa.h declares,
+and rejects bad arguments on the host before touching a GPU (no compute call is made)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import block_sparse_attention_40_b200 as qsa
+from block_sparse_attention_40_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "qsa.h")).read()
+    return sorted(set(re.findall(r"^QSA_API[^(]*?\b(qsa_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_the_bound_names():
+    assert _declared() == sorted(B.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = qsa.load()
+    for name in _declared():
+        assert hasattr(lib, name), name
+    # exported with default visibility in the dynamic symbol table
+    out = os.popen(f"nm -D --defined-only {B.library_path()}").read()
+    for name in _declared():
+        assert re.search(rf"\bT {name}\b", out), name
+
+
+def test_status_strings_and_version():
+    assert B.status_string(0) == "QSA_OK"
+    assert B.status_string(6) == "QSA_ERR_TIMEOUT"
+    assert B.status_string(99) == "QSA_ERR_UNKNOWN"
+    assert qsa.version() >= 100
+
+
+def test_workspace_sizes_grow_with_work():
+    small = B.prefill_workspace_size([0, 256], 16)
+    big = B.prefill_workspace_size([0, 65536], 512)
+    assert 0 < small < big
+    # bad lengths and budgets are rejected (size 0 -> error)
+    with pytest.raises(B.QSAError):
+        B.prefill_workspace_size([0, 0], 512)
+    with pytest.raises(B.QSAError):
+        B.prefill_workspace_size([0, 100], 0)
+    with pytest.raises(B.QSAError):
+        B.prefill_workspace_size([0, 100], 4096)
+    lib = qsa.load()
+    desc = B.CacheDesc(0, 0, 0, 0, 0, 64, 262144)
+    n = lib.qsa_decode_workspace_size(ctypes.byref(desc), B._params(512))
+    assert n > 64 * 65535 * 4
+    desc = B.CacheDesc(0, 0, 0, 0, 0, 4, 1001)   # capacity not a multiple of 4
+    assert lib.qsa_decode_workspace_size(ctypes.byref(desc), B._params(512)) == 0
+
+
+def _p(v):
+    return ctypes.c_void_p(v)
+
+
+def test_host_side_argument_errors():
+    lib = qsa.load()
+    cu = (ctypes.c_int32 * 2)(0, 64)
+    good = 0x10000
+    prm = B._params(16)
+    # null pointer
+    r = lib.qsa_prefill(None, _p(good), _p(good), _p(good), _p(good), _p(good), _p(good), cu, 1,
+                        _p(good), _p(good), 1 << 20, prm, None)
+    assert B.STATUS[r] == "QSA_ERR_INVALID_ARG"
+    # misaligned pointer
+    r = lib.qsa_prefill(_p(good + 2), _p(good), _p(good), _p(good), _p(good), _p(good), _p(good),
+                        cu, 1, _p(good), _p(good), 1 << 20, prm, None)
+    assert B.STATUS[r] == "QSA_ERR_ALIGNMENT"
+    # bad cumulative lengths
+    bad = (ctypes.c_int32 * 3)(0, 64, 60)
+    r = lib.qsa_prefill(_p(good), _p(good), _p(good), _p(good), _p(good), _p(good), _p(good), bad,
+                        2, _p(good), _p(good), 1 << 30, prm, None)
+    assert B.STATUS[r] == "QSA_ERR_INVALID_ARG"
+    # workspace too small
+    r = lib.qsa_prefill(_p(good), _p(good), _p(good), _p(good), _p(good), _p(good), _p(good), cu, 1,
+                        _p(good), _p(good), 16, prm, None)
+    assert B.STATUS[r] == "QSA_ERR_WORKSPACE"
+    # budget zero
+    r = lib.qsa_prefill(_p(good), _p(good), _p(good), _p(good), _p(good), _p(good), _p(good), cu, 1,
+                        _p(good), _p(good), 1 << 30, B._params(0), None)
+    assert B.STATUS[r] == "QSA_ERR_INVALID_ARG"
+    # append beyond capacity
+    desc = B.CacheDesc(good, good, good, good, good, 2, 64)
+    h_len = (ctypes.c_int32 * 2)(60, 10)
+    r = lib.qsa_append_kv(ctypes.byref(desc), _p(good), _p(good), _p(good), 8, None, h_len, None)
+    assert B.STATUS[r] == "QSA_ERR_CAPACITY"
+    # decode with a length of 0 (no token appended)
+    h_len = (ctypes.c_int32 * 2)(0, 10)
+    desc = B.CacheDesc(good, good, good, good, good, 2, 64)
+    r = lib.qsa_decode(_p(good), ctypes.byref(desc), _p(good), _p(good), _p(good), h_len, None,
+                       None, _p(good), 1 << 30, B._params(16), None)
+    assert B.STATUS[r] == "QSA_ERR_INVALID_ARG"
+
+
+def test_cpu_tensors_are_refused():
+    # the product has no CPU path: CPU tensors raise before any call
+    q = torch.zeros((8, 24, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        B._need(q, "q", torch.bfloat16, (24, 128), 3)

@@ -1,0 +1,116 @@
+"""GPU parity of QSA decode (append, then steps a2, a3, a6) against the oracle.
+
+The oracle evaluates the new token as row p = len-1 of the sequence made of the context
+plus every appended token (token-major), so decode is checked against the same definition
+as prefill."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import block_sparse_attention_40_b200 as qsa
+from block_sparse_attention_40_b200 import workloads as W
+from tests.gpu_helpers import compare_outputs, compare_selection, needs_gpu
+
+pytestmark = [pytest.mark.gpu, needs_gpu]
+DEV = "cuda:0"
+
+
+def _oracle_row(k_tok, v_tok, kidx_tok, q, q_idx, w, topk, forced=None):
+    """k_tok/v_tok [L,2,128], kidx_tok [L,64] (bf16 CPU), query of row L-1."""
+    L = k_tok.shape[0]
+    cu = np.array([0, L], dtype=np.int64)
+    kbar = oracle.compress(W.bits(kidx_tok), cu)
+    fi = fc = None
+    if forced is not None:
+        fi, fc = forced
+    idx, cnt, kth, out = oracle.rows(q_rows=W.bits(q[None]), q_idx_rows=W.bits(q_idx[None]),
+                                     w_rows=W.bits(w[None]), row_seq=np.zeros(1, np.int64),
+                                     row_pos=np.array([L - 1]), k=W.bits(k_tok), v=W.bits(v_tok),
+                                     kbar=kbar, cu_seqlens=cu, topk=topk, forced_idx=fi,
+                                     forced_cnt=fc)
+    return idx, cnt, kth, out, kbar
+
+
+def _decode_session(spec, check_seqs, steps, splits=0, device_gen=False):
+    gen_dev = DEV if device_gen else "cpu"
+    k_ctx, v_ctx, ki_ctx = W.decode_context(spec, device=gen_dev)
+    cache = qsa.KVCache(spec.batch, spec.capacity, DEV, zero=False)
+    # bulk fill in chunks with per-sequence counts
+    lmax = max(spec.context)
+    chunk = 16384
+    for c0 in range(0, lmax, chunk):
+        c1 = min(lmax, c0 + chunk)
+        counts = [max(0, min(c1, L) - c0) for L in spec.context]
+        cache.append(k_ctx[:, c0:c1].to(DEV), v_ctx[:, c0:c1].to(DEV), ki_ctx[:, c0:c1].to(DEV),
+                     counts=counts)
+    dec = qsa.Decoder(cache, spec.topk, splits)
+    # host copies for the oracle (only the checked sequences)
+    seqs = {b: (k_ctx[b, :spec.context[b]].cpu(), v_ctx[b, :spec.context[b]].cpu(),
+                ki_ctx[b, :spec.context[b]].cpu()) for b in check_seqs}
+    del k_ctx, v_ctx, ki_ctx
+    results = []
+    for step in range(steps):
+        st = W.decode_step(spec, step, device=gen_dev)
+        cache.append(st["k"].to(DEV), st["v"].to(DEV), st["k_idx"].to(DEV))
+        out, idx, cnt = dec.run(st["q"].to(DEV), st["q_idx"].to(DEV), st["w"].to(DEV),
+                                with_selection=True)
+        torch.cuda.synchronize()
+        assert dec.device_error() == ("QSA_OK", 0)
+        for b in check_seqs:
+            kt, vt, kit = seqs[b]
+            kt = torch.cat([kt, st["k"][b].cpu()])
+            vt = torch.cat([vt, st["v"][b].cpu()])
+            kit = torch.cat([kit, st["k_idx"][b].cpu()])
+            seqs[b] = (kt, vt, kit)
+            q, qi, w = st["q"][b].cpu(), st["q_idx"][b].cpu(), st["w"][b].cpu()
+            o_idx, o_cnt, o_kth, _, kbar = _oracle_row(kt, vt, kit, q, qi, w, spec.topk)
+            g_idx = idx[b:b + 1].cpu().numpy()
+            g_cnt = cnt[b:b + 1].cpu().numpy()
+
+            def score_fn(i, blocks, qi=qi, w=w, kbar=kbar, L=kt.shape[0]):
+                return oracle.score_pairs(W.bits(qi[None]), W.bits(w[None]), kbar,
+                                          np.array([0, L]), np.zeros(1, np.int64),
+                                          np.zeros(len(blocks), np.int64), blocks)
+
+            swaps = compare_selection(g_idx, g_cnt, o_idx, o_cnt, o_kth, score_fn)
+            _, _, _, o_out, _ = _oracle_row(kt, vt, kit, q, qi, w, spec.topk,
+                                            forced=(g_idx, g_cnt))
+            results.append((b, step, swaps) + compare_outputs(out[b:b + 1], o_out))
+            # the compressed cache agrees bit for bit with the oracle's compression
+            L = kt.shape[0]
+            got = cache.kbar[b, :L // 4].contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+            assert np.array_equal(got, kbar[:L // 4])
+    return results
+
+
+def test_small_decode_steps():
+    spec = W.small_decode_spec()
+    res = _decode_session(spec, check_seqs=[0, 1, 2, 3], steps=spec.steps)
+    assert len(res) == 4 * spec.steps
+
+
+@pytest.mark.parametrize("splits", [1, 3, 8])
+def test_small_decode_splits(splits):
+    spec = W.small_decode_spec(batch=2, context=(2045, 2046), capacity=2100, topk=128, steps=3,
+                               seed=5)
+    _decode_session(spec, check_seqs=[0, 1], steps=3, splits=splits)
+
+
+def test_decode_short_contexts():
+    # contexts shorter than the budget: decode equals dense attention over the prefix
+    spec = W.small_decode_spec(batch=4, context=(0, 1, 3, 6), capacity=64, topk=512, steps=5,
+                               seed=9)
+    _decode_session(spec, check_seqs=[0, 1, 2, 3], steps=5)
+
+
+@pytest.mark.slow
+def test_decode_256k_four_sequences():
+    spec = W.decode_spec("decode256k")
+    _decode_session(spec, check_seqs=[0, 1, 2, 3], steps=1, device_gen=True)
+
+
+@pytest.mark.slow
+def test_decode_1m_incremental():
+    spec = W.decode_spec("decode1m")
+    _decode_session(spec, check_seqs=[0, 3], steps=4, device_gen=True)

@@ -1,0 +1,88 @@
+"""GPU parity of QSA prefill (steps a1-a4) against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_40_b200 as qsa
+from block_sparse_attention_40_b200 import workloads as W
+from tests.gpu_helpers import needs_gpu, prefill_oracle_check, rows_sample
+
+pytestmark = [pytest.mark.gpu, needs_gpu]
+DEV = "cuda:0"
+
+
+def _run(p, rows_per_tile=0, chunk=0):
+    d = p.to(DEV)
+    ctx = qsa.Prefill(p.cu_seqlens, DEV, p.topk, rows_per_tile, chunk)
+    idx, cnt = ctx.select(d.q_idx, d.k_idx, d.w)
+    out = ctx.run(d.q, d.k, d.v, d.q_idx, d.k_idx, d.w)
+    torch.cuda.synchronize()
+    assert ctx.device_error() == ("QSA_OK", 0)
+    return idx, cnt, out
+
+
+def test_tiny_full():
+    p = W.prefill("tiny")
+    idx, cnt, out = _run(p)
+    res = prefill_oracle_check(p, idx, cnt, out, np.arange(256))
+    assert res["swapped_rows"] <= 2
+
+
+@pytest.mark.parametrize("rows_per_tile", [1, 3, 8, 10])
+def test_rows_per_tile_variants(rows_per_tile):
+    p = W.custom_prefill([203, 77], topk=7, kind="normal", seed=rows_per_tile)
+    idx, cnt, out = _run(p, rows_per_tile=rows_per_tile)
+    prefill_oracle_check(p, idx, cnt, out, np.arange(280))
+
+
+def test_short_sequences_and_dense_rows():
+    # lengths below one block, exactly one block, and rows whose candidates fit the budget
+    p = W.custom_prefill([1, 2, 3, 4, 5, 9, 31, 64], topk=512, kind="normal", seed=5)
+    idx, cnt, out = _run(p)
+    prefill_oracle_check(p, idx, cnt, out, np.arange(int(p.cu_seqlens[-1])))
+
+
+def test_budget_one_and_chunked_scores():
+    p = W.custom_prefill([300, 129], topk=1, kind="normal", seed=6)
+    idx, cnt, out = _run(p, chunk=48)
+    prefill_oracle_check(p, idx, cnt, out, np.arange(429))
+
+
+def test_8k_integer_selection_bit_exact():
+    p = W.prefill("8k_int")
+    d = p.to(DEV)
+    ctx = qsa.Prefill(p.cu_seqlens, DEV, p.topk)
+    idx, cnt = ctx.select(d.q_idx, d.k_idx, d.w)
+    torch.cuda.synchronize()
+    prefill_oracle_check(p, idx, cnt, None, np.arange(8192), exact_sel=True)
+
+
+def test_8k_needles_sampled():
+    p = W.prefill("8k")
+    idx, cnt, out = _run(p)
+    rows = rows_sample(8192, 1024, seed=1)
+    prefill_oracle_check(p, idx, cnt, out, rows)
+    # needles are always selected by rows that can see them
+    needles = p.needles[0]
+    ic = idx.cpu().numpy()
+    cc = cnt.cpu().numpy()
+    for t in range(0, 8192, 3):
+        sel = set(ic[t, :cc[t]].tolist())
+        assert {n for n in needles if n < t // 4} <= sel
+
+
+@pytest.mark.slow
+def test_ragged_sampled():
+    p = W.prefill("ragged")
+    idx, cnt, out = _run(p)
+    T = int(p.cu_seqlens[-1])
+    rows = rows_sample(T, 4096, seed=2, cu=p.cu_seqlens.tolist())
+    prefill_oracle_check(p, idx, cnt, out, rows)
+
+
+@pytest.mark.slow
+def test_64k_sampled():
+    p = W.prefill("64k", device=DEV)
+    idx, cnt, out = _run(p)
+    rows = rows_sample(65536, 4096, seed=3)
+    prefill_oracle_check(p, idx, cnt, out, rows)
