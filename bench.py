@@ -1,0 +1,449 @@
+#!/usr/bin/env python
+"""QSA benchmark: 64K prefill tokens/s and 256K decode tokens/s on B200, with roofline.
+
+One step = one QSA prefill of a 65,536-token sequence (budget 512 blocks; indexer keys and
+K drift per block) plus one decode step (append one token, then decode) for a batch of 64
+sequences at 262,140..262,143 tokens of context.  Inputs are seeded synthetic tensors of
+those shapes (no dataset is involved).  Each step is timed with CUDA events on the stream
+the kernels run on; L2 is flushed (a 256 MB write) before each timed part.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl qsa|reference]
+       [--workload both|prefill|decode]
+Under torchrun (N > 1) every rank runs its own replica of the step on its own GPU (the
+sequences are independent, no collective on the data path); rank 0 prints one JSON line
+with the whole-job throughput computed from the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "QSA prefill tokens/s at 64K & decode tokens/s at 256K ctx; % of roofline"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+PREFILL_T, TOPK = 65536, 512
+DEC_BATCH, DEC_CAP = 64, 262144
+
+
+# ------------------------------------------------------------------------------------
+# algorithmic work (definitions; the kernels never read these)
+def prefill_attention_flops(T=PREFILL_T, k=TOPK):
+    """Selected-token FLOPs: per token, 24 heads x 128 dims x 4 flops (QK and PV) per key."""
+    tot = 0
+    for t in range(T):
+        keys = 4 * min(k, t // 4) + (t % 4) + 1
+        tot += keys
+    return 24 * 128 * 4 * tot
+
+
+def prefill_indexer_flops(T=PREFILL_T):
+    return sum(2 * 16 * 64 * (t // 4) for t in range(T))
+
+
+def decode_bytes_per_seq(L_after, k=TOPK):
+    """HBM bytes one decode step must read/write for one sequence of L_after tokens."""
+    p = L_after - 1
+    n_c = p // 4
+    sel = min(k, n_c)
+    kbar = n_c * 64 * 2
+    kv = sel * 2 * 2 * 4 * 128 * 2               # K and V, 2 heads, 4 tokens, 128 dims
+    tail = 2 * 2 * 4 * 128 * 2                   # own block, K and V, both heads
+    q = 24 * 128 * 2 + 16 * 64 * 2 + 16 * 2      # q, q_idx, w
+    out = 24 * 128 * 2
+    append = 2 * 2 * 128 * 2 + 64 * 2            # new K, V rows and k_idx
+    return kbar + kv + tail + q + out + append
+
+
+# ------------------------------------------------------------------------------------
+def load_peaks():
+    try:
+        d = json.load(open(PEAKS_FILE))
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"qsa_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.fh,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------
+def dist_setup(n_gpus):
+    import torch
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world, device):
+    """Largest value of x across ranks (device time is taken as the slowest rank's)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------------------------
+def run_qsa(args, rank, world, local):
+    import torch
+    import block_sparse_attention_40_b200 as qsa
+    from block_sparse_attention_40_b200 import binding as B
+    from block_sparse_attention_40_b200 import workloads as W
+
+    dev = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    peaks, peak_src = load_peaks()
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def flush():
+        flush_buf.random_(0, 255)
+
+    do_prefill = args.workload in ("both", "prefill")
+    do_decode = args.workload in ("both", "decode")
+    res = {}
+
+    # ---------------- prefill setup ----------------
+    if do_prefill:
+        p = W.prefill("64k", device=dev, seed=1002 + rank)
+        ctx = qsa.Prefill(p.cu_seqlens, dev, TOPK, args.rows_per_tile, args.chunk_rows)
+        idx = torch.empty((PREFILL_T, TOPK), dtype=torch.int32, device=dev)
+        cnt = torch.empty((PREFILL_T,), dtype=torch.int32, device=dev)
+        out = torch.empty_like(p.q)
+
+    # ---------------- decode setup ----------------
+    if do_decode:
+        spec = W.decode_spec("decode256k")
+        spec.seed += 17 * rank
+        cache = qsa.KVCache(spec.batch, spec.capacity, dev, zero=False)
+        kc, vc, kic = W.decode_context(spec, device=dev)
+        lmax = max(spec.context)
+        for c0 in range(0, lmax, 16384):
+            c1 = min(lmax, c0 + 16384)
+            counts = [max(0, min(c1, L) - c0) for L in spec.context]
+            cache.append(kc[:, c0:c1].contiguous(), vc[:, c0:c1].contiguous(),
+                         kic[:, c0:c1].contiguous(), counts=counts)
+        del kc, vc, kic
+        torch.cuda.synchronize(dev)
+        torch.cuda.empty_cache()
+        saved_len = cache.len.clone()
+        saved_part = cache.kbar_partial.clone()
+        saved_hlen = list(cache.h_len)
+        dec = qsa.Decoder(cache, TOPK, args.decode_splits)
+        st = W.decode_step(spec, 0, device=dev)
+        dec_out = torch.empty_like(st["q"])
+
+        def reset_cache():
+            cache.len.copy_(saved_len)
+            cache.kbar_partial.copy_(saved_part)
+            cache.h_len = list(saved_hlen)
+
+    def step(timed, ev):
+        if do_prefill:
+            flush()
+            ev["p0"].record(stream)
+            ctx.select(p.q_idx, p.k_idx, p.w, idx, cnt)
+            ev["p1"].record(stream)
+            ctx.attend(p.q, p.k, p.v, idx, cnt, out)
+            ev["p2"].record(stream)
+        if do_decode:
+            reset_cache()
+            flush()
+            ev["d0"].record(stream)
+            cache.append(st["k"], st["v"], st["k_idx"])
+            dec.run(st["q"], st["q_idx"], st["w"], out=dec_out)
+            ev["d1"].record(stream)
+
+    names = ["p0", "p1", "p2", "d0", "d1"]
+    for _ in range(args.warmup):
+        step(False, {n: torch.cuda.Event(enable_timing=True) for n in names})
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    launches0 = B.launch_count()
+    evs = [{n: torch.cuda.Event(enable_timing=True) for n in names} for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    for i in range(args.steps):
+        step(True, evs[i])
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clk = clocks.stop()
+    launches = B.launch_count() - launches0
+    sel_ms = sum(e["p0"].elapsed_time(e["p1"]) for e in evs) if do_prefill else 0.0
+    att_ms = sum(e["p1"].elapsed_time(e["p2"]) for e in evs) if do_prefill else 0.0
+    dec_ms = sum(e["d0"].elapsed_time(e["d1"]) for e in evs) if do_decode else 0.0
+    sel_ms = max_over_ranks(sel_ms, world, dev)
+    att_ms = max_over_ranks(att_ms, world, dev)
+    dec_ms = max_over_ranks(dec_ms, world, dev)
+    K = args.steps
+    errs = []
+    if do_prefill:
+        errs.append(ctx.device_error())
+    if do_decode:
+        errs.append(dec.device_error())
+    assert all(e == ("QSA_OK", 0) for e in errs), errs
+
+    # ---------------- e2e through host buffers ----------------
+    e2e = {}
+    if args.e2e and do_prefill:
+        hp = {n: getattr(p, n).cpu().pin_memory() for n in ("q", "k", "v", "q_idx", "k_idx", "w")}
+        hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        dp = {n: torch.empty_like(getattr(p, n)) for n in hp}
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        tot = 0.0
+        for i in range(max(1, min(K, 3)) + 1):
+            flush()
+            e0.record(stream)
+            for n in hp:
+                dp[n].copy_(hp[n], non_blocking=True)
+            ctx.run(dp["q"], dp["k"], dp["v"], dp["q_idx"], dp["k_idx"], dp["w"], out)
+            hout.copy_(out, non_blocking=True)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            if i > 0:
+                tot += e0.elapsed_time(e1)
+        n_e2e = max(1, min(K, 3))
+        tot = max_over_ranks(tot, world, dev)
+        h2d = sum(t.numel() * t.element_size() for t in hp.values())
+        e2e["prefill"] = {"value": world * PREFILL_T * n_e2e / (tot / 1e3), "unit": "tokens/s",
+                          "h2d_bytes_per_step": h2d,
+                          "d2h_bytes_per_step": hout.numel() * hout.element_size()}
+        del hp, hout, dp
+    if args.e2e and do_decode:
+        hs = {n: st[n].cpu().pin_memory() for n in st}
+        ds = {n: torch.empty_like(st[n]) for n in st}
+        hout = torch.empty(dec_out.shape, dtype=dec_out.dtype, pin_memory=True)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        tot = 0.0
+        for i in range(K + 1):
+            reset_cache()
+            flush()
+            e0.record(stream)
+            for n in hs:
+                ds[n].copy_(hs[n], non_blocking=True)
+            cache.append(ds["k"], ds["v"], ds["k_idx"])
+            dec.run(ds["q"], ds["q_idx"], ds["w"], out=dec_out)
+            hout.copy_(dec_out, non_blocking=True)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            if i > 0:
+                tot += e0.elapsed_time(e1)
+        tot = max_over_ranks(tot, world, dev)
+        e2e["decode"] = {"value": world * DEC_BATCH * K / (tot / 1e3), "unit": "tokens/s",
+                         "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hs.values()),
+                         "d2h_bytes_per_step": hout.numel() * hout.element_size()}
+
+    res = dict(sel_ms=sel_ms, att_ms=att_ms, dec_ms=dec_ms, clocks=clk, launches=launches,
+               peaks=peaks, peak_src=peak_src, e2e=e2e, do_prefill=do_prefill,
+               do_decode=do_decode)
+    if do_decode:
+        res["dec_bytes"] = sum(decode_bytes_per_seq(L + 1) for L in spec.context)
+    return res
+
+
+# ------------------------------------------------------------------------------------
+def cpu_baseline(seconds_target=12.0, threads=None):
+    """The oracle, as it stands, on a bounded sample of the 64K prefill rows."""
+    import numpy as np
+    import torch
+    import oracle
+    from block_sparse_attention_40_b200 import workloads as W
+    p = W.prefill("64k", device="cpu")
+    b = {n: W.bits(getattr(p, n)) for n in ("q", "k", "v", "q_idx", "k_idx", "w")}
+    threads = threads or os.cpu_count() or 1
+    rng = np.random.default_rng(0)
+    n = 8
+    elapsed, rows_done = 0.0, 0
+    while elapsed < seconds_target and rows_done < 4096:
+        rows = np.sort(rng.integers(0, PREFILL_T, n))
+        t0 = time.perf_counter()
+        oracle.prefill(q=b["q"], k=b["k"], v=b["v"], q_idx=b["q_idx"], k_idx=b["k_idx"],
+                       w=b["w"], cu_seqlens=p.cu_seqlens.numpy().astype(np.int64), topk=TOPK,
+                       row_ids=rows, threads=threads)
+        elapsed += time.perf_counter() - t0
+        rows_done += n
+        n *= 2
+    del torch
+    return {"value": rows_done / elapsed, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{rows_done} uniformly drawn query rows of the 65,536-token prefill "
+                      f"(selection + attention per row), {elapsed:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the CPU oracle on bounded samples, timed on the host cores."""
+    if rank != 0:
+        return
+    threads = os.cpu_count() or 1
+    base = cpu_baseline(seconds_target=max(4.0, 40.0 / max(1, args.steps + args.warmup)),
+                        threads=threads)
+    line = {"impl": "reference", "metric": METRIC, "value": base["value"], "unit": "tokens/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * PREFILL_T / base["value"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "qsa_prefill_64k (oracle sample)", "seq_len": PREFILL_T,
+                       "topk_blocks": TOPK, "heads": "24q/2kv", "head_dim": 128},
+            "cpu_baseline": base,
+            "e2e": {"value": base["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["qsa", "reference"], default="qsa")
+    ap.add_argument("--workload", choices=["both", "prefill", "decode"], default="both")
+    ap.add_argument("--rows-per-tile", type=int, default=0)
+    ap.add_argument("--chunk-rows", type=int, default=0)
+    ap.add_argument("--decode-splits", type=int, default=0)
+    ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--no-cpu-baseline", dest="cpu", action="store_false")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank, world, local = dist_setup(args.gpus)
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    r = run_qsa(args, rank, world, local)
+    if rank != 0:
+        return
+    K = args.steps
+    peaks = r["peaks"]
+    line = {"metric": METRIC}
+    if r["do_prefill"]:
+        pre_ms = (r["sel_ms"] + r["att_ms"]) / K
+        attn_flops = prefill_attention_flops()
+        att_s = r["att_ms"] / K / 1e3
+        ach = attn_flops / att_s / 1e12
+        line.update({"value": world * PREFILL_T / (pre_ms / 1e3), "unit": "tokens/s"})
+        line["roofline"] = {"kernel": "qsa_sparse_attention (union plan + tcgen05 attention)",
+                            "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
+                            "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
+                            "peak_source": f"{r['peak_src']} bf16 burst",
+                            "traffic": None,
+                            "algorithmic": f"{attn_flops / 1e12:.4f} TFLOP selected-token per launch"}
+        idx_flops = prefill_indexer_flops()
+        line["prefill"] = {"tokens_per_s": world * PREFILL_T / (pre_ms / 1e3),
+                           "ms": pre_ms, "select_ms": r["sel_ms"] / K, "attention_ms": r["att_ms"] / K,
+                           "frac_of_bf16_peak_end_to_end":
+                               attn_flops / (pre_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+                           "indexer_tflop": idx_flops / 1e12,
+                           "select_tflops_indexer_only": idx_flops / (r["sel_ms"] / K / 1e3) / 1e12}
+    if r["do_decode"]:
+        dms = r["dec_ms"] / K
+        gbs = r["dec_bytes"] / (dms / 1e3) / 1e9
+        dec = {"value": world * DEC_BATCH / (dms / 1e3), "unit": "tokens/s", "ms_per_step": dms,
+               "roofline": {"kernel": "whole decode step (append, indexer, top-k, plan, "
+                                      "attention, combine)", "bound": "hbm", "achieved": gbs,
+                            "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                            "frac": gbs / peaks["hbm_gbs"],
+                            "peak_source": f"{r['peak_src']} HBM copy",
+                            "traffic": None,
+                            "algorithmic": f"{r['dec_bytes'] / 1e6:.1f} MB per step"}}
+        if "decode" in r["e2e"]:
+            dec["e2e"] = r["e2e"]["decode"]
+        line["decode"] = dec
+        if not r["do_prefill"]:
+            line.update({"value": dec["value"], "unit": "tokens/s", "roofline": dec["roofline"]})
+    ms = ((r["sel_ms"] + r["att_ms"] + r["dec_ms"]) / K)
+    line.update({"n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms,
+                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                 "dtype": "bf16", "data": "synthetic",
+                 "config": {"workload": "qsa_prefill_64k + qsa_decode_256k_b64",
+                            "prefill_seq_len": PREFILL_T, "decode_batch": DEC_BATCH,
+                            "decode_context": "262140 + (i mod 4)", "topk_blocks": TOPK,
+                            "heads": "24q/2kv", "head_dim": 128, "indexer": "16x64",
+                            "l2": "flushed (256 MB write) before each timed part",
+                            "parallelism": f"replicas x{world}"},
+                 "clocks": r["clocks"], "gpu_launches": r["launches"]})
+    if "prefill" in r["e2e"]:
+        line["e2e"] = r["e2e"]["prefill"]
+    elif "decode" in r["e2e"]:
+        line["e2e"] = r["e2e"]["decode"]
+    if args.cpu and world == 1:
+        line["cpu_baseline"] = cpu_baseline()
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

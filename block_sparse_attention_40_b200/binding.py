@@ -26,7 +26,7 @@ STATUS = {0: "QSA_OK", 1: "QSA_ERR_INVALID_ARG", 2: "QSA_ERR_ALIGNMENT", 3: "QSA
           8: "QSA_ERR_UNSUPPORTED"}
 
 # Names exported by include/qsa.h (checked by the tests).
-EXPORTS = ("qsa_status_string", "qsa_version", "qsa_workspace_init", "qsa_last_device_error",
+EXPORTS = ("qsa_status_string", "qsa_version", "qsa_launch_count", "qsa_workspace_init", "qsa_last_device_error",
            "qsa_compress_workspace_size", "qsa_compress", "qsa_index_scores", "qsa_topk",
            "qsa_prefill_workspace_size", "qsa_prefill", "qsa_prefill_select",
            "qsa_sparse_attention", "qsa_append_kv", "qsa_decode_workspace_size", "qsa_decode")
@@ -70,6 +70,7 @@ def load(build_if_needed: bool = True):
         sig = {
             "qsa_status_string": ([st], ctypes.c_char_p),
             "qsa_version": ([], I32),
+            "qsa_launch_count": ([], ctypes.c_uint64),
             "qsa_workspace_init": ([P, SZ, P], st),
             "qsa_last_device_error": ([P, P, P], st),
             "qsa_compress_workspace_size": ([I32], SZ),
@@ -161,6 +162,11 @@ def version() -> int:
     return int(load().qsa_version())
 
 
+def launch_count() -> int:
+    """Kernels launched by libqsa.so so far in this process."""
+    return int(load().qsa_launch_count())
+
+
 # --------------------------------------------------------------------------------------
 def prefill_workspace_size(cu_seqlens_host, topk=512, rows_per_tile=0, score_chunk_rows=0) -> int:
     h = torch.as_tensor(cu_seqlens_host, dtype=torch.int32).contiguous()
@@ -225,7 +231,7 @@ def index_scores(q_idx, w, kbar, cu_seqlens, row_begin=None, row_end=None, topk=
         scores = torch.full((row_end - row_begin, ld), float("nan"), dtype=torch.float32, device=dev)
     _need(scores, "scores", torch.float32)
     lib = load()
-    ws = new_workspace(prefill_workspace_size(h, max(topk, 1), 1), dev)
+    ws = new_workspace(prefill_workspace_size(h, topk if topk > 0 else 512, 1), dev)
     _check("qsa_index_scores",
            lib.qsa_index_scores(_ptr(q_idx), _ptr(w), _ptr(kbar), _ptr(d),
                                 ctypes.c_void_p(h.data_ptr()), h.numel() - 1, row_begin, row_end,

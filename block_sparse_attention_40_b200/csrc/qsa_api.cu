@@ -2,6 +2,7 @@
 // kernel launches for QSA prefill, append and decode on sm_100a.  The declarations and the
 // contract of every entry point are in include/qsa.h.
 #include <algorithm>
+#include <atomic>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -147,8 +148,11 @@ qsa_status prefill_geom(const int32_t* h_cu, int32_t num_seqs, const qsa_params&
   return QSA_OK;
 }
 
+std::atomic<uint64_t> g_launches{0};
+
 #define QSA_CHECK_LAUNCH()                                  \
   do {                                                      \
+    g_launches.fetch_add(1, std::memory_order_relaxed);     \
     cudaError_t e_ = cudaGetLastError();                    \
     if (e_ != cudaSuccess) {                                \
       fprintf(stderr, "qsa: launch failed: %s (%s:%d)\n",  \
@@ -371,6 +375,8 @@ const char* qsa_status_string(qsa_status s) {
 }
 
 int32_t qsa_version(void) { return kVersion; }
+
+uint64_t qsa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 qsa_status qsa_workspace_init(void* workspace, size_t ws_bytes, qsa_stream_t stream) {
   if (!workspace) return QSA_ERR_INVALID_ARG;

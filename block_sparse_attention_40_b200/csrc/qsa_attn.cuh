@@ -106,6 +106,7 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
   int64_t kv_row_base = 0;
   if (args.decode) {
     tok_row0 = tile;
+    pos0 = rec[2];   // p = len - 1 of the sequence
     kv_row_base = (static_cast<int64_t>(tile) * 2 + g) * args.cap_blocks * kBlock;
   } else {
     const int s = find_seq_of_tile<true>(args.meta, args.num_seqs, tile);
@@ -268,7 +269,7 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
     const int tr = row_ok ? row / kGroup : 0;
     const int hr = row % kGroup;
     const int pos = pos0 + tr;
-    const int tail_u = row_ok ? rec[2 + tr] : -1;
+    const int tail_u = row_ok ? rec[args.pl.tail_off() + tr] : -1;
     const int tail_last = pos % kBlock;   // keys 0..tail_last of the own block are visible
     const float sl2 = 1.4426950408889634f * 0.08838834764831845f;   // log2(e)/sqrt(128)
     float m = -INFINITY, l = 0.f;

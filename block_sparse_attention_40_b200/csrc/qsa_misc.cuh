@@ -437,17 +437,19 @@ struct PlanLayout {
   int32_t R;         // tokens per tile
   int32_t umax;      // union capacity per tile (multiple of 32)
   int64_t stride;    // int32 entries per tile record
-  // record: [0] = U, [1] = number of tokens, [2..2+R) = tail positions,
-  //         [2+R .. 2+R+umax) = union block ids, then R * (umax/32) mask words
-  __host__ __device__ int64_t union_off() const { return 2 + R; }
-  __host__ __device__ int64_t mask_off() const { return 2 + R + umax; }
+  // record: [0] = U, [1] = number of tokens, [2] = position of token 0 in its sequence,
+  //         [3] unused, [4..4+R) = union position of each token's own block,
+  //         [4+R .. 4+R+umax) = union block ids, then R * (umax/32) mask words
+  __host__ __device__ int64_t tail_off() const { return 4; }
+  __host__ __device__ int64_t union_off() const { return 4 + R; }
+  __host__ __device__ int64_t mask_off() const { return 4 + R + umax; }
 };
 
 __host__ __device__ inline PlanLayout make_plan_layout(int R, int topk) {
   PlanLayout pl;
   pl.R = R;
   pl.umax = ((R * (topk + 1)) + 31) / 32 * 32;
-  pl.stride = 2 + R + pl.umax + static_cast<int64_t>(R) * (pl.umax / 32);
+  pl.stride = 4 + R + pl.umax + static_cast<int64_t>(R) * (pl.umax / 32);
   pl.stride = (pl.stride + 3) / 4 * 4;   // 16-byte aligned records
   return pl;
 }
@@ -569,7 +571,7 @@ __global__ void __launch_bounds__(kPlanThreads) k_attn_plan(
         const int w = b >> 5;
         const int pos = wpref[w] + __popc(bitmap[w] & ((1u << (b & 31)) - 1u));
         atomicOr(&masks[r * mwords + (pos >> 5)], 1u << (pos & 31));
-        if (j == n) rec[2 + r] = pos;
+        if (j == n) rec[pl.tail_off() + r] = pos;
       }
     }
     __syncthreads();
@@ -582,6 +584,7 @@ __global__ void __launch_bounds__(kPlanThreads) k_attn_plan(
     if (tid == 0) {
       rec[0] = U;
       rec[1] = ntok;
+      rec[2] = pos0;
     }
     __syncthreads();
   }

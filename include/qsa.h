@@ -110,6 +110,9 @@ QSA_API const char *qsa_status_string(qsa_status s);
 /* Library version (major*10000 + minor*100 + patch). */
 QSA_API int32_t qsa_version(void);
 
+/* Number of CUDA kernels this library has launched in this process (all devices). */
+QSA_API uint64_t qsa_launch_count(void);
+
 /* Zero the status words at the start of a workspace (enqueued on stream).  Call once
  * after allocating a workspace, before its first use. */
 QSA_API qsa_status qsa_workspace_init(void *workspace, size_t ws_bytes, qsa_stream_t stream);

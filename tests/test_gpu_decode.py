@@ -42,8 +42,8 @@ def _decode_session(spec, check_seqs, steps, splits=0, device_gen=False):
     for c0 in range(0, lmax, chunk):
         c1 = min(lmax, c0 + chunk)
         counts = [max(0, min(c1, L) - c0) for L in spec.context]
-        cache.append(k_ctx[:, c0:c1].to(DEV), v_ctx[:, c0:c1].to(DEV), ki_ctx[:, c0:c1].to(DEV),
-                     counts=counts)
+        cache.append(k_ctx[:, c0:c1].to(DEV).contiguous(), v_ctx[:, c0:c1].to(DEV).contiguous(),
+                     ki_ctx[:, c0:c1].to(DEV).contiguous(), counts=counts)
     dec = qsa.Decoder(cache, spec.topk, splits)
     # host copies for the oracle (only the checked sequences)
     seqs = {b: (k_ctx[b, :spec.context[b]].cpu(), v_ctx[b, :spec.context[b]].cpu(),
