@@ -180,10 +180,14 @@ def run_qsa(args, rank, world, local):
 
     # ---------------- prefill setup ----------------
     if do_prefill:
-        p = W.prefill("64k", device=dev, seed=1002 + rank)
+        if args.prefill_len == PREFILL_T:
+            p = W.prefill("64k", device=dev, seed=1002 + rank)
+        else:   # smaller case of the same drifting workload (profiling captures)
+            p = W.custom_prefill([args.prefill_len], TOPK, kind="drift", device=dev,
+                                 seed=1002 + rank)
         ctx = qsa.Prefill(p.cu_seqlens, dev, TOPK, args.rows_per_tile, args.chunk_rows)
-        idx = torch.empty((PREFILL_T, TOPK), dtype=torch.int32, device=dev)
-        cnt = torch.empty((PREFILL_T,), dtype=torch.int32, device=dev)
+        idx = torch.empty((args.prefill_len, TOPK), dtype=torch.int32, device=dev)
+        cnt = torch.empty((args.prefill_len,), dtype=torch.int32, device=dev)
         out = torch.empty_like(p.q)
 
     # ---------------- decode setup ----------------
@@ -282,7 +286,7 @@ def run_qsa(args, rank, world, local):
         n_e2e = max(1, min(K, 3))
         tot = max_over_ranks(tot, world, dev)
         h2d = sum(t.numel() * t.element_size() for t in hp.values())
-        e2e["prefill"] = {"value": world * PREFILL_T * n_e2e / (tot / 1e3), "unit": "tokens/s",
+        e2e["prefill"] = {"value": world * args.prefill_len * n_e2e / (tot / 1e3), "unit": "tokens/s",
                           "h2d_bytes_per_step": h2d,
                           "d2h_bytes_per_step": hout.numel() * hout.element_size()}
         del hp, hout, dp
@@ -375,6 +379,8 @@ def main():
     ap.add_argument("--rows-per-tile", type=int, default=0)
     ap.add_argument("--chunk-rows", type=int, default=0)
     ap.add_argument("--decode-splits", type=int, default=0)
+    ap.add_argument("--prefill-len", type=int, default=PREFILL_T,
+                    help="prefill sequence length (default 65536; smaller only for profiling)")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu", action="store_false")
     args = ap.parse_args()
@@ -392,18 +398,18 @@ def main():
     line = {"metric": METRIC}
     if r["do_prefill"]:
         pre_ms = (r["sel_ms"] + r["att_ms"]) / K
-        attn_flops = prefill_attention_flops()
+        attn_flops = prefill_attention_flops(args.prefill_len)
         att_s = r["att_ms"] / K / 1e3
         ach = attn_flops / att_s / 1e12
-        line.update({"value": world * PREFILL_T / (pre_ms / 1e3), "unit": "tokens/s"})
+        line.update({"value": world * args.prefill_len / (pre_ms / 1e3), "unit": "tokens/s"})
         line["roofline"] = {"kernel": "qsa_sparse_attention (union plan + tcgen05 attention)",
                             "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
                             "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
                             "peak_source": f"{r['peak_src']} bf16 burst",
                             "traffic": None,
                             "algorithmic": f"{attn_flops / 1e12:.4f} TFLOP selected-token per launch"}
-        idx_flops = prefill_indexer_flops()
-        line["prefill"] = {"tokens_per_s": world * PREFILL_T / (pre_ms / 1e3),
+        idx_flops = prefill_indexer_flops(args.prefill_len)
+        line["prefill"] = {"tokens_per_s": world * args.prefill_len / (pre_ms / 1e3),
                            "ms": pre_ms, "select_ms": r["sel_ms"] / K, "attention_ms": r["att_ms"] / K,
                            "frac_of_bf16_peak_end_to_end":
                                attn_flops / (pre_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
@@ -430,7 +436,7 @@ def main():
                  "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                  "dtype": "bf16", "data": "synthetic",
                  "config": {"workload": "qsa_prefill_64k + qsa_decode_256k_b64",
-                            "prefill_seq_len": PREFILL_T, "decode_batch": DEC_BATCH,
+                            "prefill_seq_len": args.prefill_len, "decode_batch": DEC_BATCH,
                             "decode_context": "262140 + (i mod 4)", "topk_blocks": TOPK,
                             "heads": "24q/2kv", "head_dim": 128, "indexer": "16x64",
                             "l2": "flushed (256 MB write) before each timed part",
