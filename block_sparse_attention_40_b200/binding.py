@@ -29,7 +29,8 @@ STATUS = {0: "QSA_OK", 1: "QSA_ERR_INVALID_ARG", 2: "QSA_ERR_ALIGNMENT", 3: "QSA
 EXPORTS = ("qsa_status_string", "qsa_version", "qsa_launch_count", "qsa_workspace_init", "qsa_last_device_error",
            "qsa_compress_workspace_size", "qsa_compress", "qsa_index_scores", "qsa_topk",
            "qsa_prefill_workspace_size", "qsa_prefill", "qsa_prefill_select",
-           "qsa_sparse_attention", "qsa_append_kv", "qsa_decode_workspace_size", "qsa_decode")
+           "qsa_sparse_attention", "qsa_append_kv", "qsa_decode_workspace_size", "qsa_decode",
+           "qsa_decode_noalloc")
 
 
 class QSAError(RuntimeError):
@@ -84,6 +85,7 @@ def load(build_if_needed: bool = True):
             "qsa_append_kv": ([P, P, P, P, I32, P, P, P], st),
             "qsa_decode_workspace_size": ([P, Params], SZ),
             "qsa_decode": ([P, P, P, P, P, P, P, P, P, SZ, Params, P], st),
+            "qsa_decode_noalloc": ([P, P, P, P, P, P, P, P, Params, P], st),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -400,3 +402,20 @@ class Decoder:
 
     def device_error(self):
         return last_device_error(self.ws)
+
+
+def decode_noalloc(cache: KVCache, q, q_idx, w, topk=512, decode_splits=0, out=None):
+    """Decode through qsa_decode_noalloc: no workspace is passed; the library uses its own
+    fixed device scratch.  Calls must not overlap on the GPU (they share that scratch)."""
+    B = cache.batch
+    _need(q, "q", torch.bfloat16, (NUM_HEADS, HEAD_DIM), 3)
+    _need(q_idx, "q_idx", torch.bfloat16, (IDX_HEADS, IDX_DIM), 3)
+    _need(w, "w", torch.bfloat16, (IDX_HEADS,), 2)
+    if out is None:
+        out = torch.empty_like(q)
+    h_len = (ctypes.c_int32 * B)(*cache.h_len)
+    desc = cache.desc()
+    _check("qsa_decode_noalloc", load().qsa_decode_noalloc(
+        _ptr(q), ctypes.byref(desc), _ptr(q_idx), _ptr(w), _ptr(out), h_len, None, None,
+        _params(topk, 0, decode_splits, 0), _stream(q.device)))
+    return out

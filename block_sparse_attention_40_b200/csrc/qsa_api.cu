@@ -739,3 +739,53 @@ qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, 
 }
 
 }  // extern "C"
+
+// ---- decode with the library's own fixed scratch -----------------------------------------
+// One device array per GPU that loads the library, used as the workspace of
+// qsa_decode_noalloc.  In host code its name only stands for the symbol; the device
+// address comes from cudaGetSymbolAddress, looked up once per device with it current.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[QSA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+qsa_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return QSA_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return QSA_OK;
+}
+}  // namespace
+
+extern "C" qsa_status qsa_decode_noalloc(const void* q, const qsa_cache* cache, const void* q_idx,
+                                         const void* w, void* out, const int32_t* h_len,
+                                         int32_t* sel_idx, int32_t* sel_cnt, qsa_params params,
+                                         qsa_stream_t stream) {
+  if (!cache) return QSA_ERR_INVALID_ARG;
+  const size_t need = qsa_decode_workspace_size(cache, params);
+  if (need == 0) return QSA_ERR_INVALID_ARG;
+  if (need > QSA_NOALLOC_SCRATCH_BYTES) {
+    fprintf(stderr,
+            "qsa_decode_noalloc: this cache needs %zu bytes of scratch, more than the fixed "
+            "%u bytes; use qsa_decode with a workspace\n",
+            need, static_cast<unsigned>(QSA_NOALLOC_SCRATCH_BYTES));
+    return QSA_ERR_WORKSPACE;
+  }
+  void* ws = nullptr;
+  qsa_status st = noalloc_scratch(&ws);
+  if (st != QSA_OK) return st;
+  // the status words must start at zero; everything else is written before it is read
+  if (cudaMemsetAsync(ws, 0, QSA_WS_HEADER_BYTES, reinterpret_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return QSA_ERR_CUDA;
+  return qsa_decode(q, cache, q_idx, w, out, h_len, sel_idx, sel_cnt, ws,
+                    QSA_NOALLOC_SCRATCH_BYTES, params, stream);
+}

@@ -225,6 +225,33 @@ QSA_API qsa_status qsa_decode(const void *q, const qsa_cache *cache, const void 
                       void *workspace, size_t ws_bytes, qsa_params params,
                       qsa_stream_t stream);
 
+/* ---------------------------------------------------------------------------------- */
+/* Decode without a caller-provided workspace.  The pages have no counterpart of this entry
+ * point; it exists for callers that cannot allocate device memory on the call path and have
+ * no buffer to lend -- for example a plugin running inside a host framework whose allocator
+ * owns all device memory, or a serving loop that must not allocate after start-up.
+ *
+ * Same inputs, outputs and result as qsa_decode (it runs the same kernels), but the scratch
+ * lives in one fixed device array inside the library, QSA_NOALLOC_SCRATCH_BYTES (32 MiB)
+ * large, which every GPU that loads the library holds until the process exits.
+ *   - Returns QSA_ERR_WORKSPACE, with nothing enqueued, when this cache's batch, capacity
+ *     and budget need more scratch than that (compare qsa_decode_workspace_size); batch 64 at
+ *     capacity 262,144 with budget 512 needs about 19 MB.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ *   - The first call on a device looks up the array's device address with that device
+ *     current; make that first call before any stream capture.
+ *   - Every call, on every stream, shares the one array and it keeps the last call's
+ *     contents; each call clears the status words at its start.  Calls that overlap on the
+ *     GPU race on the array and corrupt each other's results: serialise them (one stream,
+ *     or events between streams).  Device-side status words of these calls cannot be read
+ *     back by the caller. */
+#define QSA_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+QSA_API qsa_status qsa_decode_noalloc(const void *q, const qsa_cache *cache, const void *q_idx,
+                                      const void *w, void *out, const int32_t *h_len,
+                                      int32_t *sel_idx, int32_t *sel_cnt, qsa_params params,
+                                      qsa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
