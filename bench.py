@@ -242,6 +242,7 @@ def run_qsa(args, rank, world, local):
     evs = [{n: torch.cuda.Event(enable_timing=True) for n in names} for _ in range(args.steps)]
     clocks = ClockSampler(local)
     clocks.start()
+    time.sleep(0.5)            # let nvidia-smi start sampling before the timed region
     torch.cuda.synchronize(dev)
     barrier(world)
     for i in range(args.steps):
@@ -372,7 +373,7 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["qsa", "reference"], default="qsa")
     ap.add_argument("--workload", choices=["both", "prefill", "decode"], default="both")

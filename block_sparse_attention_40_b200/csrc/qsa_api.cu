@@ -19,7 +19,7 @@ using namespace qsa;
 namespace {
 
 constexpr int kVersion = 100;   // 0.1.0
-constexpr int kDefaultRowsPerTile = 8;
+constexpr int kDefaultRowsPerTile = 10;
 constexpr int kDefaultScoreChunkRows = 4096;
 constexpr int kTopkSmemCap = 32768;     // row scores cached in shared memory up to this n_c
 constexpr int kNumSMsFallback = 148;

@@ -5,17 +5,20 @@
 // pairs: row = 12 * token + head, rows >= 12R are padding.  Keys are the tile's union of
 // selected blocks and own blocks (see k_attn_plan), processed 32 blocks = 128 keys per chunk.
 //
-// Per chunk i (S and P double-buffered in TMEM, K/V double-buffered in shared memory):
-//   S = Q K^T        tcgen05, A = Q (smem, K-major), B = K chunk (smem, K-major), D in TMEM
-//   softmax          one thread per row: mask keys the row's token did not select (and the
-//                    own block's future tokens), online max in the log2 domain with lazy
-//                    rescaling of O (only when the max grows by more than 2^8), P = exp2(.)
-//                    written back over S in TMEM as bf16
-//   O += P V         tcgen05, A = P (TMEM), B = V chunk (smem, MN-major), D = O in TMEM
+// Per chunk i (S and P double-buffered in TMEM; K and V in separate 3-stage shared-memory
+// rings, so K of later chunks streams in while earlier chunks are still in P.V):
+//   S = Q K^T        tcgen05, A = Q (smem, K-major), B = K chunk (smem, K-major), D in TMEM;
+//                    its completion frees the K slot
+//   softmax          one thread per row: keys of blocks the row's token did not select get
+//                    -inf (a per-block bias), and so do the own block's future tokens; online
+//                    max in the log2 domain with lazy rescaling of O (only when the max grows
+//                    by more than 2^8); P = exp2(.) written back over S in TMEM as bf16
+//   O += P V         tcgen05, A = P (TMEM), B = V chunk (smem, MN-major), D = O in TMEM;
+//                    its completion frees the V slot
 // K/V rows are gathered per 4-token block with TMA boxes of 4 rows x 64 dims (no multicast).
 //
-// Warp roles: warps 0-3 softmax (warp w owns TMEM lanes 32w..32w+31), warp 4 TMA producer,
-// warp 5 TMEM allocation + MMA issue.
+// Warp roles: warps 0-3 softmax (warp w owns TMEM lanes 32w..32w+31), warp 4 K producer,
+// warp 5 V producer, warp 6 TMEM allocation + MMA issue.
 #pragma once
 
 #include "qsa_common.cuh"
@@ -24,22 +27,24 @@
 namespace qsa {
 
 struct AttnCfg {
-  static constexpr int kThreads = 192;
+  static constexpr int kThreads = 224;
   static constexpr int kChunkBlocks = 32;
   static constexpr int kChunkKeys = 128;
-  static constexpr int kQBytes = 128 * kHeadDim * 2;     // 32 KB (2 panels of 16 KB)
-  static constexpr int kKVBytes = kChunkKeys * kHeadDim * 2;   // 32 KB per K or V tile
-  static constexpr int kStages = 2;
+  static constexpr int kQBytes = 128 * kHeadDim * 2;         // 32 KB (2 panels of 16 KB)
+  static constexpr int kKVBytes = kChunkKeys * kHeadDim * 2; // 32 KB per K or V chunk
+  static constexpr int kKStages = 3;
+  static constexpr int kVStages = 3;
   static constexpr int kQOff = 0;
-  static constexpr int kKOff = kQBytes;                        // stage s: K at kKOff + s*64KB
-  static constexpr int kStageBytes = 2 * kKVBytes;
-  static constexpr int kBarOff = kKOff + kStages * kStageBytes;
-  static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 1 + 1;
+  static constexpr int kKOff = kQBytes;
+  static constexpr int kVOff = kKOff + kKStages * kKVBytes;
+  static constexpr int kBarOff = kVOff + kVStages * kKVBytes;
+  static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 1 + 1 + 1;
   static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
-  static constexpr int kTmemCols = 512;                  // S0 [0,128) S1 [128,256) O [256,384)
+  static constexpr int kTmemCols = 512;   // S0 [0,128) S1 [128,256) O [256,384)
   static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0, 0);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 0, 1);   // B = V is MN-major
 };
+static_assert(AttnCfg::kSmemBytes <= 232448, "attention tile exceeds shared memory");
 
 struct AttnArgs {
   const int32_t* plan;     // tile records (PlanLayout)
@@ -56,13 +61,59 @@ struct AttnArgs {
   DevStatus st;
 };
 
-__device__ __forceinline__ uint32_t spread_nibbles(uint32_t byte) {
-  // bit i of byte -> nibble i of the result set to 0xF
-  uint32_t x = byte & 0xffu;
-  x = (x | (x << 12)) & 0x000F000Fu;
-  x = (x | (x << 6)) & 0x03030303u;
-  x = (x | (x << 3)) & 0x11111111u;
-  return x * 0xFu;
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  return (static_cast<uint64_t>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
+}
+__device__ __forceinline__ float f2_lo(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Producer of one operand stream (K or V) of a tile: per chunk, 32 lanes each gather one
+// 4-token block (two 128-byte-wide boxes, one per 64-dim panel).
+__device__ __forceinline__ void attn_producer(const CUtensorMap* tmap, unsigned char* ring,
+                                              uint64_t* full, uint64_t* empty, int stages,
+                                              const int32_t* uni, int U, int c_begin, int nchunks,
+                                              int64_t kv_row_base, int col0, volatile int* abort,
+                                              DevStatus st, uint32_t site) {
+  const int lane = threadIdx.x & 31;
+  int upos = c_begin * AttnCfg::kChunkBlocks + lane;
+  int blk_next = uni[upos < U ? upos : 0];
+  int issued = 0;
+  for (int i = 0; i < nchunks; ++i) {
+    const int blk = blk_next;
+    upos += AttnCfg::kChunkBlocks;
+    if (i + 1 < nchunks) blk_next = uni[upos < U ? upos : 0];   // padding repeats a real block
+    const int s = i % stages;
+    bool ok = true;
+    if (lane == 0) ok = mbar_wait(&empty[s], ((i / stages) & 1) ^ 1, abort, st, site);
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    if (!ok) break;
+    if (lane == 0) mbar_arrive_expect_tx(&full[s], AttnCfg::kKVBytes);
+    __syncwarp();
+    const int32_t row = static_cast<int32_t>(kv_row_base + static_cast<int64_t>(blk) * kBlock);
+    unsigned char* dst = ring + s * AttnCfg::kKVBytes + lane * 512;
+    tma_load_2d(dst, tmap, col0, row, &full[s]);
+    tma_load_2d(dst + 16384, tmap, col0 + 64, row, &full[s]);
+    ++issued;
+  }
+  if (lane == 0 && *abort) {
+    const int from = issued > stages ? issued - stages : 0;
+    for (int j = from; j < issued; ++j) mbar_drain(&full[j % stages], (j / stages) & 1);
+  }
 }
 
 __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
@@ -73,14 +124,20 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   unsigned char* sQ = smem + C::kQOff;
+  unsigned char* sK = smem + C::kKOff;
+  unsigned char* sV = smem + C::kVOff;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;
-  uint64_t* kv_empty = kv_full + C::kStages;
-  uint64_t* s_full = kv_empty + C::kStages;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = k_full + C::kKStages;
+  uint64_t* v_full = k_empty + C::kKStages;
+  uint64_t* v_empty = v_full + C::kVStages;
+  uint64_t* s_full = v_empty + C::kVStages;
   uint64_t* p_full = s_full + 2;
-  uint64_t* pv_done = p_full + 2;
+  uint64_t* p_free = p_full + 2;     // P.V of the buffer's last chunk has completed
+  uint64_t* pv_done = p_free + 2;
   uint64_t* mma_done = pv_done + 1;
+  uint64_t* o_final = mma_done + 1;  // every P.V of the tile has completed
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
 
@@ -133,16 +190,22 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < C::kStages; ++i) {
-      mbar_init(&kv_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+    for (int i = 0; i < C::kKStages; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < C::kVStages; ++i) {
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 4);
+      mbar_init(&p_free[i], 1);
     }
     mbar_init(pv_done, 1);
     mbar_init(mma_done, 1);
+    mbar_init(o_final, 1);
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -157,7 +220,7 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
     }
     fence_proxy_async_smem();
   }
-  if (warp == 5) {
+  if (warp == 6) {
     tmem_alloc(s_tmem, C::kTmemCols);
     tmem_relinquish();
   }
@@ -170,82 +233,61 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
   const int32_t* uni = rec + args.pl.union_off();
   const uint32_t* masks = reinterpret_cast<const uint32_t*>(rec + args.pl.mask_off());
   const int mwords = args.pl.umax / 32;
+  const int col0 = args.decode ? 0 : g * kHeadDim;
 
   if (warp == 4) {
-    // ---------------- TMA producer ----------------
+    // ---------------- Q + K producer ----------------
     if (lane == 0) {
       prefetch_tmap(&tmap_q);
       prefetch_tmap(&tmap_k);
-      prefetch_tmap(&tmap_v);
       const uint32_t qbytes = 2u * kGroup * R * 128u;   // full box, out-of-range rows zero-filled
       mbar_arrive_expect_tx(q_full, qbytes);
-      // Q box: 64 dims x 12 heads x ntok tokens, rows land as 12*token + head
       for (int half = 0; half < 2; ++half)
         tma_load_3d(sQ + half * 16384, &tmap_q, half * 64, g * kGroup,
                     static_cast<int32_t>(tok_row0), q_full);
     }
     __syncwarp();
-    int issued = 0;
-    for (int i = 0; i < nchunks; ++i) {
-      const int s = i % C::kStages;
-      bool ok = true;
-      if (lane == 0) ok = mbar_wait(&kv_empty[s], ((i / C::kStages) & 1) ^ 1, s_abort, args.st, 20);
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      if (!ok) break;
-      if (lane == 0) mbar_arrive_expect_tx(&kv_full[s], 2u * C::kKVBytes);
-      __syncwarp();
-      const int upos = (c_begin + i) * C::kChunkBlocks + lane;
-      const int blk = upos < U ? uni[upos] : uni[0];   // padding slots repeat a real block
-      unsigned char* sK = smem + C::kKOff + s * C::kStageBytes;
-      unsigned char* sV = sK + C::kKVBytes;
-      if (args.decode) {
-        const int32_t row = static_cast<int32_t>(kv_row_base + static_cast<int64_t>(blk) * kBlock);
-        for (int half = 0; half < 2; ++half) {
-          tma_load_2d(sK + half * 16384 + lane * 512, &tmap_k, half * 64, row, &kv_full[s]);
-          tma_load_2d(sV + half * 16384 + lane * 512, &tmap_v, half * 64, row, &kv_full[s]);
-        }
-      } else {
-        const int32_t row = static_cast<int32_t>(kv_row_base + static_cast<int64_t>(blk) * kBlock);
-        for (int half = 0; half < 2; ++half) {
-          tma_load_2d(sK + half * 16384 + lane * 512, &tmap_k, g * kHeadDim + half * 64, row,
-                      &kv_full[s]);
-          tma_load_2d(sV + half * 16384 + lane * 512, &tmap_v, g * kHeadDim + half * 64, row,
-                      &kv_full[s]);
-        }
-      }
-      ++issued;
-    }
-    if (lane == 0 && *s_abort) {
-      const int from = issued > C::kStages ? issued - C::kStages : 0;
-      for (int j = from; j < issued; ++j) mbar_drain(&kv_full[j % C::kStages], (j / C::kStages) & 1);
-      mbar_drain(q_full, 0);
-    }
+    attn_producer(&tmap_k, sK, k_full, k_empty, C::kKStages, uni, U, c_begin, nchunks,
+                  kv_row_base, col0, s_abort, args.st, 20);
+    if (lane == 0 && *s_abort) mbar_drain(q_full, 0);
   } else if (warp == 5) {
+    // ---------------- V producer ----------------
+    if (lane == 0) prefetch_tmap(&tmap_v);
+    __syncwarp();
+    attn_producer(&tmap_v, sV, v_full, v_empty, C::kVStages, uni, U, c_begin, nchunks,
+                  kv_row_base, col0, s_abort, args.st, 27);
+  } else if (warp == 6) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       const uint32_t sQ0 = smem_u32(sQ);
       bool ok = mbar_wait(q_full, 0, s_abort, args.st, 21);
       auto issue_pv = [&](int j) -> bool {
         const int bj = j & 1;
+        const int vs = j % C::kVStages;
         if (!mbar_wait(&p_full[bj], (j >> 1) & 1, s_abort, args.st, 22)) return false;
+        if (!mbar_wait(&v_full[vs], (j / C::kVStages) & 1, s_abort, args.st, 28)) return false;
         tc_fence_after();
-        const uint32_t sV0 = smem_u32(smem + C::kKOff + (j % C::kStages) * C::kStageBytes + C::kKVBytes);
+        const uint32_t sV0 = smem_u32(sV + vs * C::kKVBytes);
 #pragma unroll
         for (int k = 0; k < C::kChunkKeys / 16; ++k) {
           // B = V chunk, MN-major: 16 keys per step = 2048 bytes; next 64 dims at +16 KB
           const uint64_t db = smem_desc_sw128(sV0 + 2048 * k, 16384, 1024);
           umma_ts(tmem_O, tmem + bj * 128 + 8 * k, db, C::kIdescPV, (j > 0 || k > 0) ? 1u : 0u);
         }
-        umma_commit(&kv_empty[j % C::kStages]);
+        umma_commit(&v_empty[vs]);
+        umma_commit(&p_free[bj]);
         umma_commit(pv_done);
         return true;
       };
       for (int i = 0; ok && i < nchunks; ++i) {
         const int b = i & 1;
-        const int s = i % C::kStages;
-        if (!mbar_wait(&kv_full[s], (i / C::kStages) & 1, s_abort, args.st, 23)) break;
+        const int ks = i % C::kKStages;
+        if (!mbar_wait(&k_full[ks], (i / C::kKStages) & 1, s_abort, args.st, 23)) break;
+        // S_i overwrites the TMEM buffer that held P_{i-2}: P_{i-2}.V must have completed
+        // (tcgen05 MMAs in flight are not ordered against each other's TMEM accesses)
+        if (i >= 2 && !mbar_wait(&p_free[b], ((i - 2) >> 1) & 1, s_abort, args.st, 29)) break;
         tc_fence_after();
-        const uint32_t sK0 = smem_u32(smem + C::kKOff + s * C::kStageBytes);
+        const uint32_t sK0 = smem_u32(sK + ks * C::kKVBytes);
 #pragma unroll
         for (int k = 0; k < kHeadDim / 16; ++k) {
           const int half = k >> 2, kk = k & 3;
@@ -253,9 +295,10 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
           const uint64_t db = smem_desc_sw128(sK0 + half * 16384 + 32 * kk, 0, 1024);
           umma_ss(tmem + b * 128, da, db, C::kIdescQK, k > 0 ? 1u : 0u);
         }
+        umma_commit(&k_empty[ks]);
         umma_commit(&s_full[b]);
         if (i > 0 && !issue_pv(i - 1)) break;
-        if (i == nchunks - 1) issue_pv(i);
+        if (i == nchunks - 1 && issue_pv(i)) umma_commit(o_final);
       }
       umma_commit(mma_done);
       mbar_drain(mma_done, 0);
@@ -269,14 +312,19 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
     const int tr = row_ok ? row / kGroup : 0;
     const int hr = row % kGroup;
     const int pos = pos0 + tr;
-    const int tail_u = row_ok ? rec[args.pl.tail_off() + tr] : -1;
+    const int tail_u = row_ok ? rec[args.pl.tail_off() + tr] : -1000000;
     const int tail_last = pos % kBlock;   // keys 0..tail_last of the own block are visible
     const float sl2 = 1.4426950408889634f * 0.08838834764831845f;   // log2(e)/sqrt(128)
     float m = -INFINITY, l = 0.f;
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t* mrow = masks + tr * mwords;
+    uint32_t mword_next = row_ok ? mrow[c_begin] : 0u;
     bool ok = true;
     for (int i = 0; i < nchunks; ++i) {
       const int b = i & 1;
+      const int q = c_begin + i;
+      const uint32_t mword = mword_next;
+      if (row_ok && i + 1 < nchunks) mword_next = mrow[q + 1];
       const bool got = mbar_wait(&s_full[b], (i >> 1) & 1, s_abort, args.st, 24);
       if (__any_sync(0xffffffffu, !got)) {   // also reconverges the warp
         ok = false;
@@ -284,82 +332,91 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
       }
       tc_fence_after();
       if (warp_active) {
-        const int q = c_begin + i;
-        uint32_t mword = row_ok ? masks[tr * mwords + q] : 0u;
-        uint32_t km[4];
-#pragma unroll
-        for (int w4 = 0; w4 < 4; ++w4) km[w4] = spread_nibbles(mword >> (8 * w4));
-        const int tu = tail_u - q * C::kChunkBlocks;
-        if (tu >= 0 && tu < C::kChunkBlocks) {
-          // hide the own block's keys after the query position
-          const int key0 = tu * 4;
-          for (int kk = tail_last + 1; kk < 4; ++kk) {
-            const int key = key0 + kk;
-            km[key >> 5] &= ~(1u << (key & 31));
-          }
-        }
         uint32_t sv[128];
         const uint32_t ts = tmem + lane_base + b * 128;
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32(ts + 32 * c, sv + 32 * c);
         tmem_wait_ld();
-        float mx = -INFINITY;
+        // keys of blocks this row's token did not select -> -inf
 #pragma unroll
-        for (int j = 0; j < 128; ++j) {
-          const bool v = (km[j >> 5] >> (j & 31)) & 1u;
-          const float x = v ? __uint_as_float(sv[j]) * sl2 : -INFINITY;
-          sv[j] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
+        for (int u = 0; u < 32; ++u) {
+          const float bias = ((mword >> u) & 1u) ? 0.f : -INFINITY;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            sv[4 * u + kk] = __float_as_uint(__uint_as_float(sv[4 * u + kk]) + bias);
         }
-        const float m_cand = fmaxf(m, mx);
-        const bool need = m_cand > m + 8.f || (m == -INFINITY && m_cand > -INFINITY);
-        if (__any_sync(0xffffffffu, need)) {
-          const float alpha = (m == -INFINITY) ? 0.f : exp2f(m - m_cand);
-          if (i > 0) {
-            // O holds PV of chunks < i-1 and maybe i-1: wait until chunk i-1 is in, rescale
-            if (!mbar_wait(pv_done, (i - 1) & 1, s_abort, args.st, 25)) {
-              ok = false;
-            }
-            if (__any_sync(0xffffffffu, !ok)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t to = tmem_O + lane_base;
+        // the own block: hide the tokens after the query (only in the chunk holding it)
+        const int tu = tail_u - q * C::kChunkBlocks;
+        if (__any_sync(0xffffffffu, tu >= 0 && tu < C::kChunkBlocks)) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              uint32_t ov[32];
-              tmem_ld32(to + 32 * c, ov);
-              tmem_wait_ld();
-#pragma unroll
-              for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
-              tmem_st32(to + 32 * c, ov);
+          for (int u = 0; u < 32; ++u) {
+            if (u == tu) {
+              if (tail_last < 1) sv[4 * u + 1] = __float_as_uint(-INFINITY);
+              if (tail_last < 2) sv[4 * u + 2] = __float_as_uint(-INFINITY);
+              if (tail_last < 3) sv[4 * u + 3] = __float_as_uint(-INFINITY);
             }
           }
-          l *= alpha;
+        }
+        float mxs[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) mxs[j] = __uint_as_float(sv[j]);
+#pragma unroll
+        for (int j = 8; j < 128; ++j) mxs[j & 7] = fmaxf(mxs[j & 7], __uint_as_float(sv[j]));
+        const float mx = fmaxf(fmaxf(fmaxf(mxs[0], mxs[1]), fmaxf(mxs[2], mxs[3])),
+                               fmaxf(fmaxf(mxs[4], mxs[5]), fmaxf(mxs[6], mxs[7])));
+        const float m_cand = fmaxf(m, mx * sl2);
+        const bool need = m_cand > m + 8.f || (m == -INFINITY && m_cand > -INFINITY);
+        const bool rescale = __any_sync(0xffffffffu, need);
+        float alpha = 1.f;
+        if (rescale) {
+          alpha = (m == -INFINITY) ? 0.f : ex2_approx(m - m_cand);
           m = m_cand;
         }
-        const float mref = (m == -INFINITY) ? 0.f : m;
-        float lsum = 0.f;
-        uint32_t pk[64];
+        const float mneg = (m == -INFINITY) ? 0.f : -m;
+        // P overwrites S in registers: packed pair j lands in sv[j], whose S value (key j) was
+        // consumed at pair j/2 <= j
+        float lsum[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int j = 0; j < 64; ++j) {
-          const float p0 = exp2f(__uint_as_float(sv[2 * j]) - mref);
-          const float p1 = exp2f(__uint_as_float(sv[2 * j + 1]) - mref);
-          lsum += p0 + p1;
-          pk[j] = pack_bf16x2(p0, p1);
+          const float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * j]), sl2, mneg));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * j + 1]), sl2, mneg));
+          lsum[j & 3] += p0 + p1;
+          sv[j] = pack_bf16x2(p0, p1);
         }
-        l += lsum;
-        tmem_st32(ts, pk);
-        tmem_st32(ts + 32, pk + 32);
+        l = l * alpha + ((lsum[0] + lsum[1]) + (lsum[2] + lsum[3]));
+        tmem_st32(ts, sv);
+        tmem_st32(ts + 32, sv + 32);
         tmem_wait_st();
+        if (rescale && i > 0) {
+          // O holds P.V of chunks < i-1 and maybe i-1: wait until chunk i-1 is in, rescale.
+          // P.V of chunk i cannot start before this warp arrives on p_full below.
+          const bool gotpv = mbar_wait(pv_done, (i - 1) & 1, s_abort, args.st, 25);
+          if (__any_sync(0xffffffffu, !gotpv)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t to = tmem_O + lane_base;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t ov[32];
+            tmem_ld32(to + 32 * c, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
+            tmem_st32(to + 32 * c, ov);
+          }
+          tmem_wait_st();
+        }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[b]);
     }
     if (ok && nchunks > 0) {
-      const bool got = mbar_wait(pv_done, (nchunks - 1) & 1, s_abort, args.st, 26);
+      // a dedicated barrier: two P.V may still be in flight here, so a parity wait on
+      // pv_done could match an older phase
+      const bool got = mbar_wait(o_final, 0, s_abort, args.st, 26);
       if (!__any_sync(0xffffffffu, !got)) {
         tc_fence_after();
         if (warp_active) {
@@ -399,7 +456,7 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 6) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
