@@ -20,7 +20,7 @@ namespace {
 
 constexpr int kVersion = 100;   // 0.1.0
 constexpr int kDefaultRowsPerTile = 10;
-constexpr int kDefaultScoreChunkRows = 4096;
+constexpr int kDefaultScoreChunkRows = 16384;
 constexpr int kTopkSmemCap = 32768;     // row scores cached in shared memory up to this n_c
 constexpr int kNumSMsFallback = 148;
 
@@ -190,14 +190,28 @@ qsa_status launch_compress(const void* k_idx, const SeqMeta* meta, int num_seqs,
   return QSA_OK;
 }
 
+// Top-k over `rows` score rows.  Rows longer than the shared-memory cache take their first
+// radix digit from a multi-CTA histogram when `hist` (rows x 4096 uint32 of scratch) is given.
 qsa_status launch_topk(const float* scores, int64_t ld, const int32_t* n_c, int64_t rows,
-                       int topk, int max_nc, int32_t* idx, int32_t* cnt, cudaStream_t s) {
+                       int topk, int max_nc, int32_t* idx, int32_t* cnt, cudaStream_t s,
+                       uint32_t* hist = nullptr) {
   if (rows <= 0) return QSA_OK;
   const int cap = std::min(max_nc, kTopkSmemCap);
-  const int smem = 2048 * 4 + 64 * 4 + std::max(cap, 0) * 4;
+  const int smem = kTopkSharedBytes + std::max(cap, 0) * 4;
   if (!set_smem(k_topk, smem)) return QSA_ERR_CUDA;
+  const uint32_t* h1 = nullptr;
+  if (hist && max_nc > cap) {
+    if (cudaMemsetAsync(hist, 0, static_cast<size_t>(rows) * kTopkBins * 4, s) != cudaSuccess)
+      return QSA_ERR_CUDA;
+    int parts = static_cast<int>(std::max<int64_t>(1, (4 * num_sms() + rows - 1) / rows));
+    parts = std::min(parts, std::max(1, max_nc / 4096));
+    k_topk_hist<<<static_cast<int>(rows * parts), kTopkThreads, 0, s>>>(scores, ld, n_c, topk,
+                                                                         parts, hist);
+    QSA_CHECK_LAUNCH();
+    h1 = hist;
+  }
   const int grid = static_cast<int>(std::min<int64_t>(rows, int64_t(num_sms()) * 8));
-  k_topk<<<grid, kTopkThreads, smem, s>>>(scores, ld, n_c, rows, topk, cap, idx, cnt);
+  k_topk<<<grid, kTopkThreads, smem, s>>>(scores, ld, n_c, rows, topk, cap, h1, idx, cnt);
   QSA_CHECK_LAUNCH();
   return QSA_OK;
 }
@@ -323,7 +337,7 @@ struct DecodeGeom {
   int64_t ld = 4;
   PlanLayout pl;
   size_t o_scores = 0, o_nc = 0, o_idx = 0, o_cnt = 0, o_plan = 0, o_po = 0, o_pm = 0, o_pl = 0,
-         total = 0;
+         o_hist = 0, total = 0;
 };
 
 qsa_status decode_geom(const qsa_cache* c, const qsa_params& p, DecodeGeom* g) {
@@ -350,6 +364,7 @@ qsa_status decode_geom(const qsa_cache* c, const qsa_params& p, DecodeGeom* g) {
   g->o_po = cv.take(parts * kHeadDim * 4);
   g->o_pm = cv.take(parts * 4);
   g->o_pl = cv.take(parts * 4);
+  g->o_hist = cv.take(static_cast<size_t>(g->B) * kTopkBins * 4);
   g->total = cv.off;
   return QSA_OK;
 }
@@ -691,7 +706,8 @@ qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, 
     QSA_CHECK_LAUNCH();
   }
   // a3: top-k
-  st = launch_topk(scores, g.ld, n_c, g.B, g.topk, max_nc_now, idx, cnt, s);
+  st = launch_topk(scores, g.ld, n_c, g.B, g.topk, max_nc_now, idx, cnt, s,
+                   reinterpret_cast<uint32_t*>(ws + g.o_hist));
   if (st != QSA_OK) return st;
   // union plan (one token per tile)
   {

@@ -323,23 +323,159 @@ __global__ void k_append_len(int32_t* len, const int32_t* counts, int32_t n_new,
 }
 
 // ---------------------------------------------------------------------------------------
-// Step a3: top-k per row by radix select on order-preserving uint32 keys (11+11+10 bits),
-// then an ordered compaction that emits the selected blocks in ascending index order and
-// breaks ties at the threshold toward lower indices.  One 512-thread CTA per row.
+// Step a3: top-k per row by radix select on order-preserving uint32 keys, digits of 12, 12
+// and 8 bits, then an ordered compaction that emits the selected blocks in ascending index
+// order and breaks ties at the threshold toward lower indices.  One 512-thread CTA per row;
+// a row of at most `smem_cap` scores is first copied to shared memory.  When `hist1` is
+// given (long decode rows), the first-digit histogram was built by k_topk_hist across many
+// CTAs and is read from there.
 constexpr int kTopkThreads = 512;
+constexpr int kTopkWarps = kTopkThreads / 32;
+constexpr int kTopkBins = 4096;
 
-__device__ __forceinline__ float topk_load(const float* src, int i) { return src[i]; }
+struct TopkShared {
+  uint32_t hist[kTopkBins];
+  int sh[40];
+  int sel[2];
+  int wgt[kTopkWarps];
+  int weq[kTopkWarps];
+};
+// Byte offset of the cached score row in k_topk's dynamic shared memory (16-byte aligned for
+// the float4 copy; the host sizes the allocation with the same constant).
+constexpr int kTopkSharedBytes = (static_cast<int>(sizeof(TopkShared)) + 127) / 128 * 128;
 
-__global__ void __launch_bounds__(kTopkThreads) k_topk(const float* __restrict__ scores,
-                                                       int64_t ld, const int32_t* __restrict__ n_c,
-                                                       int64_t rows, int topk, int smem_cap,
+// Find the bin where the count of keys in higher bins first reaches `need` (bins scanned
+// from the top).  Returns the bin; *above receives the count of keys in higher bins.
+__device__ __forceinline__ int topk_find_bin(TopkShared& S, int nbins, int need, int* above) {
+  const int tid = threadIdx.x;
+  const int per = nbins / kTopkThreads;   // 8 or 1 (or 0: only the first threads)
+  int local = 0;
+  int lo_bin = 0, hi_bin = -1;
+  if (per > 0) {
+    hi_bin = nbins - 1 - tid * per;       // thread 0 owns the highest bins
+    lo_bin = hi_bin - per + 1;
+  } else if (tid < nbins) {
+    hi_bin = lo_bin = nbins - 1 - tid;
+  }
+  for (int b = hi_bin; b >= lo_bin; --b) local += static_cast<int>(S.hist[b]);
+  int tot;
+  const int ex = block_excl_scan(local, S.sh, &tot);   // keys in bins above my range
+  int running = ex;
+  for (int b = hi_bin; b >= lo_bin; --b) {
+    const int h = static_cast<int>(S.hist[b]);
+    if (running < need && running + h >= need) {
+      S.sel[0] = b;
+      S.sel[1] = running;
+    }
+    running += h;
+  }
+  __syncthreads();
+  *above = S.sel[1];
+  const int bin = S.sel[0];
+  __syncthreads();
+  return bin;
+}
+
+__device__ __forceinline__ void topk_row(const float* __restrict__ src, int n, int topk,
+                                         const uint32_t* hist1, int32_t* __restrict__ out,
+                                         TopkShared& S) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int need = topk;
+  // ---- digit 1: key bits [31:20] ----
+  if (hist1) {
+    for (int i = tid; i < kTopkBins; i += kTopkThreads) S.hist[i] = hist1[i];
+  } else {
+    for (int i = tid; i < kTopkBins; i += kTopkThreads) S.hist[i] = 0;
+    __syncthreads();
+    for (int base = 0; base < n; base += kTopkThreads) {
+      const int i = base + tid;
+      const uint32_t bin = i < n ? (float_key(src[i]) >> 20) : 0xffffffffu;
+      const unsigned act = __ballot_sync(0xffffffffu, i < n);
+      if (i < n) {
+        const unsigned peers = __match_any_sync(act, bin);   // lanes sharing this bin
+        if (lane == __ffs(peers) - 1) atomicAdd(&S.hist[bin], static_cast<uint32_t>(__popc(peers)));
+      }
+    }
+  }
+  __syncthreads();
+  int above;
+  const uint32_t b1 = static_cast<uint32_t>(topk_find_bin(S, kTopkBins, need, &above));
+  need -= above;
+  // ---- digit 2: bits [19:8] among keys in bin b1 ----
+  for (int i = tid; i < kTopkBins; i += kTopkThreads) S.hist[i] = 0;
+  __syncthreads();
+  for (int i = tid; i < n; i += kTopkThreads) {
+    const uint32_t key = float_key(src[i]);
+    if ((key >> 20) == b1) atomicAdd(&S.hist[(key >> 8) & 0xfffu], 1u);
+  }
+  __syncthreads();
+  const uint32_t b2 = static_cast<uint32_t>(topk_find_bin(S, kTopkBins, need, &above));
+  need -= above;
+  // ---- digit 3: bits [7:0] ----
+  const uint32_t pre = (b1 << 12) | b2;
+  for (int i = tid; i < 256; i += kTopkThreads) S.hist[i] = 0;
+  __syncthreads();
+  for (int i = tid; i < n; i += kTopkThreads) {
+    const uint32_t key = float_key(src[i]);
+    if ((key >> 8) == pre) atomicAdd(&S.hist[key & 0xffu], 1u);
+  }
+  __syncthreads();
+  const uint32_t b3 = static_cast<uint32_t>(topk_find_bin(S, 256, need, &above));
+  need -= above;
+  const uint32_t T = (pre << 8) | b3;   // the k-th largest key
+  const int need_eq = need;             // keys equal to T to take, lowest indices first
+  // ---- ordered output: each warp owns a contiguous segment ----
+  const int seg = ((n + kTopkWarps - 1) / kTopkWarps + 31) / 32 * 32;
+  const int s0 = warp * seg;
+  const int s1 = min(n, s0 + seg);
+  int c_gt = 0, c_eq = 0;
+  for (int base = s0; base < s1; base += 32) {
+    const int i = base + lane;
+    const uint32_t key = i < s1 ? float_key(src[i]) : 0u;
+    c_gt += __popc(__ballot_sync(0xffffffffu, i < s1 && key > T));
+    c_eq += __popc(__ballot_sync(0xffffffffu, i < s1 && key == T));
+  }
+  if (lane == 0) {
+    S.wgt[warp] = c_gt;
+    S.weq[warp] = c_eq;
+  }
+  __syncthreads();
+  int eq_before = 0, out_before = 0;
+  for (int w = 0; w < warp; ++w) {
+    const int eqw = S.weq[w];
+    const int takew = min(max(need_eq - eq_before, 0), eqw);
+    out_before += S.wgt[w] + takew;
+    eq_before += eqw;
+  }
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int base = s0; base < s1; base += 32) {
+    const int i = base + lane;
+    const uint32_t key = i < s1 ? float_key(src[i]) : 0u;
+    const bool gt = i < s1 && key > T;
+    const bool eq = i < s1 && key == T;
+    const unsigned eqm = __ballot_sync(0xffffffffu, eq);
+    const int eq_rank = eq_before + __popc(eqm & lt_mask);
+    const bool take = gt || (eq && eq_rank < need_eq);
+    const unsigned tm = __ballot_sync(0xffffffffu, take);
+    if (take) {
+      const int pos = out_before + __popc(tm & lt_mask);
+      if (pos < topk) out[pos] = i;
+    }
+    out_before += __popc(tm);
+    eq_before += __popc(eqm);
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kTopkThreads) k_topk(const float* __restrict__ scores, int64_t ld,
+                                                       const int32_t* __restrict__ n_c, int64_t rows,
+                                                       int topk, int smem_cap,
+                                                       const uint32_t* __restrict__ hist1,
                                                        int32_t* __restrict__ idx,
                                                        int32_t* __restrict__ cnt) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw);          // 2048
-  int* sh = reinterpret_cast<int*>(hist + 2048);                     // 33 (+ pad)
-  int* sel = sh + 40;                                                // 2
-  float* row_cache = reinterpret_cast<float*>(smem_raw + 2048 * 4 + 64 * 4);
+  TopkShared& S = *reinterpret_cast<TopkShared*>(smem_raw);
+  float* row_cache = reinterpret_cast<float*>(smem_raw + kTopkSharedBytes);
   const int tid = threadIdx.x;
   for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
     const int n = n_c[r];
@@ -351,80 +487,47 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float* __restrict__
     }
     const float* src = scores + r * ld;
     if (n <= smem_cap) {
-      for (int i = tid; i < n; i += blockDim.x) row_cache[i] = src[i];
+      const int n4 = n >> 2;
+      const float4* s4 = reinterpret_cast<const float4*>(src);
+      for (int i = tid; i < n4; i += blockDim.x) reinterpret_cast<float4*>(row_cache)[i] = s4[i];
+      for (int i = 4 * n4 + tid; i < n; i += blockDim.x) row_cache[i] = src[i];
       src = row_cache;
       __syncthreads();
     }
-    uint32_t prefix = 0, pmask = 0;
-    int need = topk;
-    const int shifts[3] = {21, 10, 0};
-    const int bitsv[3] = {11, 11, 10};
-    for (int pass = 0; pass < 3; ++pass) {
-      const int shift = shifts[pass];
-      const int nbins = 1 << bitsv[pass];
-      const uint32_t bmask = static_cast<uint32_t>(nbins - 1);
-      for (int i = tid; i < 2048; i += blockDim.x) hist[i] = 0;
-      __syncthreads();
-      for (int i = tid; i < n; i += blockDim.x) {
-        const uint32_t key = float_key(src[i]);
-        if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & bmask], 1u);
-      }
-      __syncthreads();
-      // suffix scan over bins (from the highest bin down)
-      const int per = nbins / kTopkThreads;   // 4 or 2
-      const int rt = kTopkThreads - 1 - tid;  // thread owning the highest bins has rt = 0
-      const int b_hi = (tid + 1) * per - 1;   // my highest bin
-      int local = 0;
-      for (int q = 0; q < per; ++q) local += static_cast<int>(hist[b_hi - q]);
-      int tot;
-      // exclusive scan in rt order == sum over threads with higher tid
-      // (threads are reordered through the rt index)
-      __shared__ int sh_rt[kTopkThreads];
-      sh_rt[rt] = local;
-      __syncthreads();
-      const int v = sh_rt[tid];   // value of the thread whose rt == tid
-      const int ex = block_excl_scan(v, sh, &tot);
-      sh_rt[tid] = ex;            // exclusive prefix for rt == tid
-      __syncthreads();
-      int running = sh_rt[rt];
-      for (int q = 0; q < per; ++q) {
-        const int bin = b_hi - q;
-        const int h = static_cast<int>(hist[bin]);
-        if (running < need && running + h >= need) {
-          sel[0] = bin;
-          sel[1] = running;
-        }
-        running += h;
-      }
-      __syncthreads();
-      const int bin = sel[0];
-      need -= sel[1];
-      prefix |= static_cast<uint32_t>(bin) << shift;
-      pmask |= bmask << shift;
-      __syncthreads();
-    }
-    const uint32_t T = prefix;
-    const int need_eq = need;   // elements equal to T to take (lowest indices first)
-    int base_out = 0, eq_seen = 0;
-    for (int start = 0; start < n; start += blockDim.x) {
-      const int i = start + tid;
-      uint32_t key = 0;
-      if (i < n) key = float_key(src[i]);
-      const int gt = (i < n && key > T) ? 1 : 0;
-      const int eq = (i < n && key == T) ? 1 : 0;
-      int eq_tot;
-      const int eq_rank = eq_seen + block_excl_scan(eq, sh, &eq_tot);
-      const int take = (gt || (eq && eq_rank < need_eq)) ? 1 : 0;
-      int take_tot;
-      const int pos = base_out + block_excl_scan(take, sh, &take_tot);
-      if (take && pos < topk) out[pos] = i;
-      base_out += take_tot;
-      eq_seen += eq_tot;
-      if (base_out >= topk) break;
-    }
+    topk_row(src, n, topk, hist1 ? hist1 + r * kTopkBins : nullptr, out, S);
     if (tid == 0) cnt[r] = topk;
-    __syncthreads();
   }
+}
+
+// First-digit histograms of long rows, split over `parts` CTAs per row (global atomics into
+// hist [rows][4096], which the caller zeroes).  Rows with n_c <= topk are skipped.
+__global__ void __launch_bounds__(kTopkThreads) k_topk_hist(const float* __restrict__ scores,
+                                                            int64_t ld, const int32_t* __restrict__ n_c,
+                                                            int topk, int parts,
+                                                            uint32_t* __restrict__ hist) {
+  __shared__ uint32_t h[kTopkBins];
+  const int r = blockIdx.x / parts, part = blockIdx.x % parts;
+  const int n = n_c[r];
+  if (n <= topk) return;
+  const int lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kTopkBins; i += blockDim.x) h[i] = 0;
+  __syncthreads();
+  const int per = (n + parts - 1) / parts;
+  const int a = part * per, b = min(n, a + per);
+  const float* src = scores + static_cast<int64_t>(r) * ld;
+  for (int base = a; base < b; base += kTopkThreads) {
+    const int i = base + threadIdx.x;
+    const uint32_t bin = i < b ? (float_key(src[i]) >> 20) : 0xffffffffu;
+    const unsigned act = __ballot_sync(0xffffffffu, i < b);
+    if (i < b) {
+      const unsigned peers = __match_any_sync(act, bin);
+      if (lane == __ffs(peers) - 1) atomicAdd(&h[bin], static_cast<uint32_t>(__popc(peers)));
+    }
+  }
+  __syncthreads();
+  uint32_t* dst = hist + static_cast<int64_t>(r) * kTopkBins;
+  for (int i = threadIdx.x; i < kTopkBins; i += blockDim.x)
+    if (h[i]) atomicAdd(&dst[i], h[i]);
 }
 
 // ---------------------------------------------------------------------------------------
