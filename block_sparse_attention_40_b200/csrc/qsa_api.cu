@@ -293,22 +293,23 @@ qsa_status run_attention(const void* q, const void* k, const void* v, const int3
                                                         dev_status(ws));
     QSA_CHECK_LAUNCH();
   }
-  CUtensorMap tm_q, tm_k, tm_v;
+  AttnMaps maps;
   {
     const uint64_t dims[3] = {128, 24, static_cast<uint64_t>(g.T)};
     const uint64_t strides[2] = {256, 24 * 256};
     const uint32_t box[3] = {64, 12, static_cast<uint32_t>(g.R)};
-    if (!make_tmap(&tm_q, q, 3, dims, strides, box)) return QSA_ERR_CUDA;
+    if (!make_tmap(&maps.q, q, 3, dims, strides, box)) return QSA_ERR_CUDA;
   }
-  {
+  for (int j = 0; j < kNumBoxSizes; ++j) {
     const uint64_t dims[2] = {256, static_cast<uint64_t>(g.T)};
     const uint64_t strides[1] = {512};
-    const uint32_t box[2] = {64, 4};
-    if (!make_tmap(&tm_k, k, 2, dims, strides, box)) return QSA_ERR_CUDA;
-    if (!make_tmap(&tm_v, v, 2, dims, strides, box)) return QSA_ERR_CUDA;
+    const uint32_t box[2] = {64, 4u << j};
+    if (!make_tmap(&maps.k[j], k, 2, dims, strides, box)) return QSA_ERR_CUDA;
+    if (!make_tmap(&maps.v[j], v, 2, dims, strides, box)) return QSA_ERR_CUDA;
   }
   if (!set_smem(k_sparse_attn, AttnCfg::kSmemBytes)) return QSA_ERR_CUDA;
   AttnArgs a{};
+  a.oob_row = static_cast<int32_t>(g.T);
   a.plan = plan;
   a.pl = g.pl;
   a.meta = meta;
@@ -318,7 +319,7 @@ qsa_status run_attention(const void* q, const void* k, const void* v, const int3
   a.out = reinterpret_cast<__nv_bfloat16*>(out);
   a.st = dev_status(ws);
   dim3 grid(g.attn_tiles, 2, 1);
-  k_sparse_attn<<<grid, AttnCfg::kThreads, AttnCfg::kSmemBytes, s>>>(tm_q, tm_k, tm_v, a);
+  k_sparse_attn<<<grid, AttnCfg::kThreads, AttnCfg::kSmemBytes, s>>>(maps, a);
   QSA_CHECK_LAUNCH();
   return QSA_OK;
 }
@@ -721,18 +722,22 @@ qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, 
   }
   // a6: split attention + combine
   {
-    CUtensorMap tm_q, tm_k, tm_v;
+    AttnMaps maps;
     const uint64_t dq[3] = {128, 24, static_cast<uint64_t>(g.B)};
     const uint64_t sq[2] = {256, 24 * 256};
     const uint32_t bq[3] = {64, 12, 1};
-    if (!make_tmap(&tm_q, q, 3, dq, sq, bq)) return QSA_ERR_CUDA;
+    if (!make_tmap(&maps.q, q, 3, dq, sq, bq)) return QSA_ERR_CUDA;
     const uint64_t dkv[2] = {128, static_cast<uint64_t>(g.B) * 2 * g.cap};
     const uint64_t skv[1] = {256};
-    const uint32_t bkv[2] = {64, 4};
-    if (!make_tmap(&tm_k, cache->k_blocks, 2, dkv, skv, bkv)) return QSA_ERR_CUDA;
-    if (!make_tmap(&tm_v, cache->v_blocks, 2, dkv, skv, bkv)) return QSA_ERR_CUDA;
+    for (int j = 0; j < kNumBoxSizes; ++j) {
+      const uint32_t bkv[2] = {64, 4u << j};
+      if (!make_tmap(&maps.k[j], cache->k_blocks, 2, dkv, skv, bkv)) return QSA_ERR_CUDA;
+      if (!make_tmap(&maps.v[j], cache->v_blocks, 2, dkv, skv, bkv)) return QSA_ERR_CUDA;
+    }
     if (!set_smem(k_sparse_attn, AttnCfg::kSmemBytes)) return QSA_ERR_CUDA;
     AttnArgs a{};
+    if (static_cast<uint64_t>(g.B) * 2 * g.cap >= 0x7fffffffull) return QSA_ERR_UNSUPPORTED;
+    a.oob_row = static_cast<int32_t>(static_cast<int64_t>(g.B) * 2 * g.cap);
     a.plan = plan;
     a.pl = g.pl;
     a.decode = 1;
@@ -743,7 +748,7 @@ qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, 
     a.part_l = reinterpret_cast<float*>(ws + g.o_pl);
     a.st = dev_status(ws);
     dim3 grid(g.B, 2, g.splits);
-    k_sparse_attn<<<grid, AttnCfg::kThreads, AttnCfg::kSmemBytes, s>>>(tm_q, tm_k, tm_v, a);
+    k_sparse_attn<<<grid, AttnCfg::kThreads, AttnCfg::kSmemBytes, s>>>(maps, a);
     QSA_CHECK_LAUNCH();
     const int warps = g.B * kHeads;
     k_decode_combine<<<(warps * 32 + 255) / 256, 256, 0, s>>>(a.part_o, a.part_m, a.part_l, g.B,

@@ -15,7 +15,8 @@
 //                    by more than 2^8); P = exp2(.) written back over S in TMEM as bf16
 //   O += P V         tcgen05, A = P (TMEM), B = V chunk (smem, MN-major), D = O in TMEM;
 //                    its completion frees the V slot
-// K/V rows are gathered per 4-token block with TMA boxes of 4 rows x 64 dims (no multicast).
+// K/V rows are gathered with TMA boxes of 4..128 rows x 64 dims, one per power-of-two piece of
+// each run of consecutive blocks (no multicast).
 //
 // Warp roles: warps 0-3 softmax (warp w owns TMEM lanes 32w..32w+31), warp 4 K producer,
 // warp 5 V producer, warp 6 TMEM allocation + MMA issue.
@@ -46,8 +47,19 @@ struct AttnCfg {
 };
 static_assert(AttnCfg::kSmemBytes <= 232448, "attention tile exceeds shared memory");
 
+// Tensor maps of one attention launch.  K and V each have six maps whose boxes are 64 dims
+// wide and 4, 8, 16, 32, 64, 128 rows high (1..32 consecutive blocks), so that a run of
+// consecutive selected blocks is gathered with a few large boxes instead of one per block.
+constexpr int kNumBoxSizes = 6;
+struct AttnMaps {
+  CUtensorMap q;
+  CUtensorMap k[kNumBoxSizes];
+  CUtensorMap v[kNumBoxSizes];
+};
+
 struct AttnArgs {
   const int32_t* plan;     // tile records (PlanLayout)
+  int32_t oob_row;         // a K/V row index past the end of the tensor (zero-filled by TMA)
   PlanLayout pl;
   const SeqMeta* meta;     // prefill
   int32_t num_seqs;
@@ -82,21 +94,24 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// Producer of one operand stream (K or V) of a tile: per chunk, 32 lanes each gather one
-// 4-token block (two 128-byte-wide boxes, one per 64-dim panel).
-__device__ __forceinline__ void attn_producer(const CUtensorMap* tmap, unsigned char* ring,
+// Producer of one operand stream (K or V) of a tile.  Lane u of the warp owns union slot u of
+// the chunk.  Maximal runs of consecutive block ids (and the run of padding slots past the
+// end of the union) are cut into power-of-two pieces; the first lane of each run issues one
+// TMA box per piece (rows 4*blk.., two 64-dim panels).  Padding rows come from an
+// out-of-range coordinate and are zero-filled.
+__device__ __forceinline__ void attn_producer(const CUtensorMap* maps, unsigned char* ring,
                                               uint64_t* full, uint64_t* empty, int stages,
                                               const int32_t* uni, int U, int c_begin, int nchunks,
-                                              int64_t kv_row_base, int col0, volatile int* abort,
-                                              DevStatus st, uint32_t site) {
+                                              int64_t kv_row_base, int col0, int32_t oob_row,
+                                              volatile int* abort, DevStatus st, uint32_t site) {
   const int lane = threadIdx.x & 31;
   int upos = c_begin * AttnCfg::kChunkBlocks + lane;
-  int blk_next = uni[upos < U ? upos : 0];
+  int blk_next = upos < U ? uni[upos] : -1;
   int issued = 0;
   for (int i = 0; i < nchunks; ++i) {
-    const int blk = blk_next;
+    const int blk = blk_next;           // -1: padding slot
     upos += AttnCfg::kChunkBlocks;
-    if (i + 1 < nchunks) blk_next = uni[upos < U ? upos : 0];   // padding repeats a real block
+    if (i + 1 < nchunks) blk_next = upos < U ? uni[upos] : -1;
     const int s = i % stages;
     bool ok = true;
     if (lane == 0) ok = mbar_wait(&empty[s], ((i / stages) & 1) ^ 1, abort, st, site);
@@ -104,10 +119,31 @@ __device__ __forceinline__ void attn_producer(const CUtensorMap* tmap, unsigned 
     if (!ok) break;
     if (lane == 0) mbar_arrive_expect_tx(&full[s], AttnCfg::kKVBytes);
     __syncwarp();
-    const int32_t row = static_cast<int32_t>(kv_row_base + static_cast<int64_t>(blk) * kBlock);
-    unsigned char* dst = ring + s * AttnCfg::kKVBytes + lane * 512;
-    tma_load_2d(dst, tmap, col0, row, &full[s]);
-    tma_load_2d(dst + 16384, tmap, col0 + 64, row, &full[s]);
+    const int prev = __shfl_up_sync(0xffffffffu, blk, 1);
+    const bool start = lane == 0 || (blk < 0) != (prev < 0) || (blk >= 0 && blk != prev + 1);
+    const unsigned starts = __ballot_sync(0xffffffffu, start);
+    if (start) {
+      const unsigned later = starts & ~((2u << lane) - 1u);   // run starts after this lane
+      const int run_end = later ? __ffs(later) - 1 : 32;
+      int off = 0;
+      while (off < run_end - lane) {
+        const int rem = run_end - lane - off;
+        const int slot = lane + off;
+        // the largest power of two that fits the rest of the run and divides the slot: every
+        // box starts in shared memory at a multiple of its own size (>= 512 bytes)
+        const int lg_fit = 31 - __clz(rem);
+        const int lg_align = slot == 0 ? 5 : __ffs(slot) - 1;
+        const int lg = lg_fit < lg_align ? lg_fit : lg_align;
+        const int32_t row = blk < 0 ? oob_row
+                                    : static_cast<int32_t>(kv_row_base +
+                                                           static_cast<int64_t>(blk + off) * kBlock);
+        unsigned char* dst = ring + s * AttnCfg::kKVBytes + slot * 512;
+        tma_load_2d(dst, &maps[lg], col0, row, &full[s]);
+        tma_load_2d(dst + 16384, &maps[lg], col0 + 64, row, &full[s]);
+        off += 1 << lg;
+      }
+    }
+    __syncwarp();
     ++issued;
   }
   if (lane == 0 && *abort) {
@@ -117,8 +153,7 @@ __device__ __forceinline__ void attn_producer(const CUtensorMap* tmap, unsigned 
 }
 
 __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
-    k_sparse_attn(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
-                  const __grid_constant__ CUtensorMap tmap_v, AttnArgs args) {
+    k_sparse_attn(const __grid_constant__ AttnMaps maps, AttnArgs args) {
   using C = AttnCfg;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -238,24 +273,25 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
   if (warp == 4) {
     // ---------------- Q + K producer ----------------
     if (lane == 0) {
-      prefetch_tmap(&tmap_q);
-      prefetch_tmap(&tmap_k);
+      prefetch_tmap(&maps.q);
+      for (int j = 0; j < kNumBoxSizes; ++j) prefetch_tmap(&maps.k[j]);
       const uint32_t qbytes = 2u * kGroup * R * 128u;   // full box, out-of-range rows zero-filled
       mbar_arrive_expect_tx(q_full, qbytes);
       for (int half = 0; half < 2; ++half)
-        tma_load_3d(sQ + half * 16384, &tmap_q, half * 64, g * kGroup,
+        tma_load_3d(sQ + half * 16384, &maps.q, half * 64, g * kGroup,
                     static_cast<int32_t>(tok_row0), q_full);
     }
     __syncwarp();
-    attn_producer(&tmap_k, sK, k_full, k_empty, C::kKStages, uni, U, c_begin, nchunks,
-                  kv_row_base, col0, s_abort, args.st, 20);
+    attn_producer(maps.k, sK, k_full, k_empty, C::kKStages, uni, U, c_begin, nchunks,
+                  kv_row_base, col0, args.oob_row, s_abort, args.st, 20);
     if (lane == 0 && *s_abort) mbar_drain(q_full, 0);
   } else if (warp == 5) {
     // ---------------- V producer ----------------
-    if (lane == 0) prefetch_tmap(&tmap_v);
+    if (lane == 0)
+      for (int j = 0; j < kNumBoxSizes; ++j) prefetch_tmap(&maps.v[j]);
     __syncwarp();
-    attn_producer(&tmap_v, sV, v_full, v_empty, C::kVStages, uni, U, c_begin, nchunks,
-                  kv_row_base, col0, s_abort, args.st, 27);
+    attn_producer(maps.v, sV, v_full, v_empty, C::kVStages, uni, U, c_begin, nchunks,
+                  kv_row_base, col0, args.oob_row, s_abort, args.st, 27);
   } else if (warp == 6) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
