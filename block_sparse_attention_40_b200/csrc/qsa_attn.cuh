@@ -5,8 +5,8 @@
 // pairs: row = 12 * token + head, rows >= 12R are padding.  Keys are the tile's union of
 // selected blocks and own blocks (see k_attn_plan), processed 32 blocks = 128 keys per chunk.
 //
-// Per chunk i (S and P double-buffered in TMEM; K and V in separate 3-stage shared-memory
-// rings, so K of later chunks streams in while earlier chunks are still in P.V):
+// Per chunk i (S and P double-buffered in TMEM; K and V in separate shared-memory rings of 3
+// and 2 stages, so K of later chunks streams in while earlier chunks are still in P.V):
 //   S = Q K^T        tcgen05, A = Q (smem, K-major), B = K chunk (smem, K-major), D in TMEM;
 //                    its completion frees the K slot
 //   softmax          one thread per row: keys of blocks the row's token did not select get
@@ -15,11 +15,12 @@
 //                    by more than 2^8); P = exp2(.) written back over S in TMEM as bf16
 //   O += P V         tcgen05, A = P (TMEM), B = V chunk (smem, MN-major), D = O in TMEM;
 //                    its completion frees the V slot
-// K/V rows are gathered with TMA boxes of 4..128 rows x 64 dims, one per power-of-two piece of
-// each run of consecutive blocks (no multicast).
+// K/V rows are gathered with TMA boxes of 4..128 rows x 64 dims, one per naturally aligned
+// power-of-two piece of each run of consecutive blocks (no multicast).
 //
-// Warp roles: warps 0-3 softmax (warp w owns TMEM lanes 32w..32w+31), warp 4 K producer,
-// warp 5 V producer, warp 6 TMEM allocation + MMA issue.
+// Warp roles: warps 0-7 softmax (warp w owns TMEM lanes 32(w%4)..+31; warps 0-3 handle keys
+// 0-63 of each chunk, warps 4-7 keys 64-127), warp 8 Q+K producer, warp 9 V producer,
+// warp 10 TMEM allocation + MMA issue.
 #pragma once
 
 #include "qsa_common.cuh"
@@ -28,17 +29,19 @@
 namespace qsa {
 
 struct AttnCfg {
-  static constexpr int kThreads = 224;
+  static constexpr int kThreads = 352;   // 8 softmax warps, K and V producers, MMA
   static constexpr int kChunkBlocks = 32;
   static constexpr int kChunkKeys = 128;
   static constexpr int kQBytes = 128 * kHeadDim * 2;         // 32 KB (2 panels of 16 KB)
   static constexpr int kKVBytes = kChunkKeys * kHeadDim * 2; // 32 KB per K or V chunk
   static constexpr int kKStages = 3;
-  static constexpr int kVStages = 3;
+  static constexpr int kVStages = 2;
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQBytes;
   static constexpr int kVOff = kKOff + kKStages * kKVBytes;
-  static constexpr int kBarOff = kVOff + kVStages * kKVBytes;
+  static constexpr int kXOff = kVOff + kVStages * kKVBytes;    // row-max / row-sum exchange
+  static constexpr int kXBytes = (2 * 2 * 128 + 2 * 128) * 4;
+  static constexpr int kBarOff = kXOff + kXBytes;
   static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 1 + 1 + 1;
   static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
   static constexpr int kTmemCols = 512;   // S0 [0,128) S1 [128,256) O [256,384)
@@ -161,6 +164,8 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
   unsigned char* sQ = smem + C::kQOff;
   unsigned char* sK = smem + C::kKOff;
   unsigned char* sV = smem + C::kVOff;
+  float* xmax = reinterpret_cast<float*>(smem + C::kXOff);   // [parity][wg][128]
+  float* xsum = xmax + 2 * 2 * 128;                           // [wg][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
@@ -235,7 +240,7 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 4);
+      mbar_init(&p_full[i], 8);
       mbar_init(&p_free[i], 1);
     }
     mbar_init(pv_done, 1);
@@ -255,7 +260,7 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
     }
     fence_proxy_async_smem();
   }
-  if (warp == 6) {
+  if (warp == 10) {
     tmem_alloc(s_tmem, C::kTmemCols);
     tmem_relinquish();
   }
@@ -270,7 +275,7 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
   const int mwords = args.pl.umax / 32;
   const int col0 = args.decode ? 0 : g * kHeadDim;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ---------------- Q + K producer ----------------
     if (lane == 0) {
       prefetch_tmap(&maps.q);
@@ -285,14 +290,14 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
     attn_producer(maps.k, sK, k_full, k_empty, C::kKStages, uni, U, c_begin, nchunks,
                   kv_row_base, col0, args.oob_row, s_abort, args.st, 20);
     if (lane == 0 && *s_abort) mbar_drain(q_full, 0);
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ---------------- V producer ----------------
     if (lane == 0)
       for (int j = 0; j < kNumBoxSizes; ++j) prefetch_tmap(&maps.v[j]);
     __syncwarp();
     attn_producer(maps.v, sV, v_full, v_empty, C::kVStages, uni, U, c_begin, nchunks,
                   kv_row_base, col0, args.oob_row, s_abort, args.st, 27);
-  } else if (warp == 6) {
+  } else if (warp == 10) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       const uint32_t sQ0 = smem_u32(sQ);
@@ -340,11 +345,17 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
       mbar_drain(mma_done, 0);
     }
   } else {
-    // ---------------- softmax (warps 0-3) ----------------
-    const int row = warp * 32 + lane;
+    // ---------------- softmax (warps 0-7) ----------------
+    // Two warpgroups share each row: warpgroup wg handles keys [64 wg, 64 wg + 64) of every
+    // chunk and dims [64 wg, 64 wg + 64) of O.  Row maxima are exchanged through shared memory
+    // (double-buffered by chunk parity, one named barrier per chunk); partial row sums are
+    // combined once at the end.  Both halves take identical rescale decisions.
+    const int wg = warp >> 2;
+    const int quarter = warp & 3;           // TMEM lanes 32q .. 32q+31
+    const int row = quarter * 32 + lane;
     const int valid_rows = kGroup * ntok;
     const bool row_ok = row < valid_rows;
-    const bool warp_active = warp * 32 < valid_rows;
+    const bool warp_active = quarter * 32 < valid_rows;
     const int tr = row_ok ? row / kGroup : 0;
     const int hr = row % kGroup;
     const int pos = pos0 + tr;
@@ -352,40 +363,38 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
     const int tail_last = pos % kBlock;   // keys 0..tail_last of the own block are visible
     const float sl2 = 1.4426950408889634f * 0.08838834764831845f;   // log2(e)/sqrt(128)
     float m = -INFINITY, l = 0.f;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t* mrow = masks + tr * mwords;
     uint32_t mword_next = row_ok ? mrow[c_begin] : 0u;
     bool ok = true;
     for (int i = 0; i < nchunks; ++i) {
       const int b = i & 1;
       const int q = c_begin + i;
-      const uint32_t mword = mword_next;
+      const uint32_t mword = (mword_next >> (16 * wg)) & 0xffffu;   // my 16 blocks
       if (row_ok && i + 1 < nchunks) mword_next = mrow[q + 1];
-      const bool got = mbar_wait(&s_full[b], (i >> 1) & 1, s_abort, args.st, 24);
-      if (__any_sync(0xffffffffu, !got)) {   // also reconverges the warp
-        ok = false;
-        break;
-      }
+      bool got = ok ? mbar_wait(&s_full[b], (i >> 1) & 1, s_abort, args.st, 24) : false;
+      if (__any_sync(0xffffffffu, !got)) ok = false;   // also reconverges the warp
       tc_fence_after();
-      if (warp_active) {
-        uint32_t sv[128];
-        const uint32_t ts = tmem + lane_base + b * 128;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(ts + 32 * c, sv + 32 * c);
+      uint32_t sv[64];
+      const uint32_t ts = tmem + lane_base + b * 128;
+      float mx = -INFINITY;
+      if (ok && warp_active) {
+        tmem_ld32(ts + 64 * wg, sv);
+        tmem_ld32(ts + 64 * wg + 32, sv + 32);
         tmem_wait_ld();
         // keys of blocks this row's token did not select -> -inf
 #pragma unroll
-        for (int u = 0; u < 32; ++u) {
+        for (int u = 0; u < 16; ++u) {
           const float bias = ((mword >> u) & 1u) ? 0.f : -INFINITY;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             sv[4 * u + kk] = __float_as_uint(__uint_as_float(sv[4 * u + kk]) + bias);
         }
-        // the own block: hide the tokens after the query (only in the chunk holding it)
-        const int tu = tail_u - q * C::kChunkBlocks;
-        if (__any_sync(0xffffffffu, tu >= 0 && tu < C::kChunkBlocks)) {
+        // the own block: hide the tokens after the query (only where it lies)
+        const int tu = tail_u - q * C::kChunkBlocks - 16 * wg;
+        if (__any_sync(0xffffffffu, tu >= 0 && tu < 16)) {
 #pragma unroll
-          for (int u = 0; u < 32; ++u) {
+          for (int u = 0; u < 16; ++u) {
             if (u == tu) {
               if (tail_last < 1) sv[4 * u + 1] = __float_as_uint(-INFINITY);
               if (tail_last < 2) sv[4 * u + 2] = __float_as_uint(-INFINITY);
@@ -397,9 +406,17 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
 #pragma unroll
         for (int j = 0; j < 8; ++j) mxs[j] = __uint_as_float(sv[j]);
 #pragma unroll
-        for (int j = 8; j < 128; ++j) mxs[j & 7] = fmaxf(mxs[j & 7], __uint_as_float(sv[j]));
-        const float mx = fmaxf(fmaxf(fmaxf(mxs[0], mxs[1]), fmaxf(mxs[2], mxs[3])),
-                               fmaxf(fmaxf(mxs[4], mxs[5]), fmaxf(mxs[6], mxs[7])));
+        for (int j = 8; j < 64; ++j) mxs[j & 7] = fmaxf(mxs[j & 7], __uint_as_float(sv[j]));
+        mx = fmaxf(fmaxf(fmaxf(mxs[0], mxs[1]), fmaxf(mxs[2], mxs[3])),
+                   fmaxf(fmaxf(mxs[4], mxs[5]), fmaxf(mxs[6], mxs[7])));
+      }
+      // exchange the half-row maxima (every softmax warp takes part, active or not)
+      xmax[(b * 2 + wg) * 128 + row] = mx;
+      tc_fence_before();
+      named_barrier_sync(1, 256);
+      tc_fence_after();
+      if (ok && warp_active) {
+        mx = fmaxf(mx, xmax[(b * 2 + (wg ^ 1)) * 128 + row]);
         const float m_cand = fmaxf(m, mx * sl2);
         const bool need = m_cand > m + 8.f || (m == -INFINITY && m_cand > -INFINITY);
         const bool rescale = __any_sync(0xffffffffu, need);
@@ -413,42 +430,46 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
         // consumed at pair j/2 <= j
         float lsum[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
+        for (int j = 0; j < 32; ++j) {
           const float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * j]), sl2, mneg));
           const float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * j + 1]), sl2, mneg));
           lsum[j & 3] += p0 + p1;
           sv[j] = pack_bf16x2(p0, p1);
         }
         l = l * alpha + ((lsum[0] + lsum[1]) + (lsum[2] + lsum[3]));
-        tmem_st32(ts, sv);
-        tmem_st32(ts + 32, sv + 32);
+        // packed P of keys 64 wg .. 64 wg + 63 -> columns 32 wg .. 32 wg + 31 of the buffer
+        // (the other half's S there was loaded before the barrier above)
+        tmem_st32(ts + 32 * wg, sv);
         tmem_wait_st();
         if (rescale && i > 0) {
-          // O holds P.V of chunks < i-1 and maybe i-1: wait until chunk i-1 is in, rescale.
-          // P.V of chunk i cannot start before this warp arrives on p_full below.
+          // O holds P.V of chunks < i-1 and maybe i-1: wait until chunk i-1 is in, rescale
+          // my half of O.  P.V of chunk i cannot start before this warp arrives on p_full.
           const bool gotpv = mbar_wait(pv_done, (i - 1) & 1, s_abort, args.st, 25);
-          if (__any_sync(0xffffffffu, !gotpv)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t to = tmem_O + lane_base;
+          if (__any_sync(0xffffffffu, !gotpv)) ok = false;
+          if (ok) {
+            tc_fence_after();
+            const uint32_t to = tmem_O + lane_base + 64 * wg;
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t ov[32];
-            tmem_ld32(to + 32 * c, ov);
-            tmem_wait_ld();
+            for (int c = 0; c < 2; ++c) {
+              uint32_t ov[32];
+              tmem_ld32(to + 32 * c, ov);
+              tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
-            tmem_st32(to + 32 * c, ov);
+              for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
+              tmem_st32(to + 32 * c, ov);
+            }
+            tmem_wait_st();
           }
-          tmem_wait_st();
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[b]);
     }
+    // combine the half-row sums
+    xsum[wg * 128 + row] = l;
+    named_barrier_sync(1, 256);
+    const float l_all = l + xsum[(wg ^ 1) * 128 + row];
     if (ok && nchunks > 0) {
       // a dedicated barrier: two P.V may still be in flight here, so a parity wait on
       // pv_done could match an older phase
@@ -456,17 +477,18 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
       if (!__any_sync(0xffffffffu, !got)) {
         tc_fence_after();
         if (warp_active) {
-          const uint32_t to = tmem_O + lane_base;
-          uint32_t ov[128];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) tmem_ld32(to + 32 * c, ov + 32 * c);
+          const uint32_t to = tmem_O + lane_base + 64 * wg;
+          uint32_t ov[64];
+          tmem_ld32(to, ov);
+          tmem_ld32(to + 32, ov + 32);
           tmem_wait_ld();
           if (row_ok) {
             if (!args.decode) {
-              const float inv = l > 0.f ? 1.f / l : 0.f;
-              __nv_bfloat16* o = args.out + ((tok_row0 + tr) * kHeads + g * kGroup + hr) * kHeadDim;
+              const float inv = l_all > 0.f ? 1.f / l_all : 0.f;
+              __nv_bfloat16* o = args.out + ((tok_row0 + tr) * kHeads + g * kGroup + hr) * kHeadDim +
+                                 64 * wg;
 #pragma unroll
-              for (int c = 0; c < 16; ++c) {
+              for (int c = 0; c < 8; ++c) {
                 uint4 v;
                 v.x = pack_bf16x2(__uint_as_float(ov[8 * c + 0]) * inv, __uint_as_float(ov[8 * c + 1]) * inv);
                 v.y = pack_bf16x2(__uint_as_float(ov[8 * c + 2]) * inv, __uint_as_float(ov[8 * c + 3]) * inv);
@@ -477,11 +499,13 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
             } else {
               const int64_t pr =
                   ((static_cast<int64_t>(tile) * 2 + g) * args.splits + split) * kGroup + hr;
-              args.part_m[pr] = m;
-              args.part_l[pr] = l;
-              float4* po = reinterpret_cast<float4*>(args.part_o + pr * kHeadDim);
+              if (wg == 0) {
+                args.part_m[pr] = m;
+                args.part_l[pr] = l_all;
+              }
+              float4* po = reinterpret_cast<float4*>(args.part_o + pr * kHeadDim + 64 * wg);
 #pragma unroll
-              for (int c = 0; c < 32; ++c)
+              for (int c = 0; c < 16; ++c)
                 po[c] = make_float4(__uint_as_float(ov[4 * c]), __uint_as_float(ov[4 * c + 1]),
                                     __uint_as_float(ov[4 * c + 2]), __uint_as_float(ov[4 * c + 3]));
             }
@@ -492,7 +516,7 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 6) {
+  if (warp == 10) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
