@@ -194,6 +194,9 @@ def run_qsa(args, rank, world, local):
     if do_decode:
         spec = W.decode_spec("decode256k")
         spec.seed += 17 * rank
+        if args.decode_batch != spec.batch:   # smaller case of the same workload (captures)
+            spec.batch = args.decode_batch
+            spec.context = [262140 + (i % 4) for i in range(spec.batch)]
         cache = qsa.KVCache(spec.batch, spec.capacity, dev, zero=False)
         kc, vc, kic = W.decode_context(spec, device=dev)
         lmax = max(spec.context)
@@ -311,7 +314,7 @@ def run_qsa(args, rank, world, local):
             if i > 0:
                 tot += e0.elapsed_time(e1)
         tot = max_over_ranks(tot, world, dev)
-        e2e["decode"] = {"value": world * DEC_BATCH * K / (tot / 1e3), "unit": "tokens/s",
+        e2e["decode"] = {"value": world * args.decode_batch * K / (tot / 1e3), "unit": "tokens/s",
                          "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hs.values()),
                          "d2h_bytes_per_step": hout.numel() * hout.element_size()}
 
@@ -380,6 +383,8 @@ def main():
     ap.add_argument("--rows-per-tile", type=int, default=0)
     ap.add_argument("--chunk-rows", type=int, default=0)
     ap.add_argument("--decode-splits", type=int, default=0)
+    ap.add_argument("--decode-batch", type=int, default=DEC_BATCH,
+                    help="sequences of the 256K-context decode batch (64 = the workload)")
     ap.add_argument("--prefill-len", type=int, default=PREFILL_T,
                     help="prefill sequence length (default 65536; smaller only for profiling)")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
@@ -419,7 +424,7 @@ def main():
     if r["do_decode"]:
         dms = r["dec_ms"] / K
         gbs = r["dec_bytes"] / (dms / 1e3) / 1e9
-        dec = {"value": world * DEC_BATCH / (dms / 1e3), "unit": "tokens/s", "ms_per_step": dms,
+        dec = {"value": world * args.decode_batch / (dms / 1e3), "unit": "tokens/s", "ms_per_step": dms,
                "roofline": {"kernel": "whole decode step (append, indexer, top-k, plan, "
                                       "attention, combine)", "bound": "hbm", "achieved": gbs,
                             "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -436,8 +441,10 @@ def main():
     line.update({"n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms,
                  "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                  "dtype": "bf16", "data": "synthetic",
-                 "config": {"workload": "qsa_prefill_64k + qsa_decode_256k_b64",
-                            "prefill_seq_len": args.prefill_len, "decode_batch": DEC_BATCH,
+                 "config": {"workload": " + ".join(
+                                ([f"qsa_prefill_{args.prefill_len // 1024}k"] if r["do_prefill"] else [])
+                                + ([f"qsa_decode_256k_b{args.decode_batch}"] if r["do_decode"] else [])),
+                            "prefill_seq_len": args.prefill_len, "decode_batch": args.decode_batch,
                             "decode_context": "262140 + (i mod 4)", "topk_blocks": TOPK,
                             "heads": "24q/2kv", "head_dim": 128, "indexer": "16x64",
                             "l2": "flushed (256 MB write) before each timed part",

@@ -22,6 +22,7 @@ constexpr int kVersion = 100;   // 0.1.0
 constexpr int kDefaultRowsPerTile = 10;
 constexpr int kDefaultScoreChunkRows = 16384;
 constexpr int kTopkSmemCap = 32768;     // row scores cached in shared memory up to this n_c
+constexpr int kCandCap = 16384;         // decode top-k candidates per row
 constexpr int kNumSMsFallback = 148;
 
 // ---- driver entry point for tensor-map encoding (no link-time libcuda dependency) ----
@@ -190,28 +191,15 @@ qsa_status launch_compress(const void* k_idx, const SeqMeta* meta, int num_seqs,
   return QSA_OK;
 }
 
-// Top-k over `rows` score rows.  Rows longer than the shared-memory cache take their first
-// radix digit from a multi-CTA histogram when `hist` (rows x 4096 uint32 of scratch) is given.
+// Top-k over `rows` score rows (one CTA per row; short rows cached in shared memory).
 qsa_status launch_topk(const float* scores, int64_t ld, const int32_t* n_c, int64_t rows,
-                       int topk, int max_nc, int32_t* idx, int32_t* cnt, cudaStream_t s,
-                       uint32_t* hist = nullptr) {
+                       int topk, int max_nc, int32_t* idx, int32_t* cnt, cudaStream_t s) {
   if (rows <= 0) return QSA_OK;
   const int cap = std::min(max_nc, kTopkSmemCap);
   const int smem = kTopkSharedBytes + std::max(cap, 0) * 4;
   if (!set_smem(k_topk, smem)) return QSA_ERR_CUDA;
-  const uint32_t* h1 = nullptr;
-  if (hist && max_nc > cap) {
-    if (cudaMemsetAsync(hist, 0, static_cast<size_t>(rows) * kTopkBins * 4, s) != cudaSuccess)
-      return QSA_ERR_CUDA;
-    int parts = static_cast<int>(std::max<int64_t>(1, (4 * num_sms() + rows - 1) / rows));
-    parts = std::min(parts, std::max(1, max_nc / 4096));
-    k_topk_hist<<<static_cast<int>(rows * parts), kTopkThreads, 0, s>>>(scores, ld, n_c, topk,
-                                                                         parts, hist);
-    QSA_CHECK_LAUNCH();
-    h1 = hist;
-  }
   const int grid = static_cast<int>(std::min<int64_t>(rows, int64_t(num_sms()) * 8));
-  k_topk<<<grid, kTopkThreads, smem, s>>>(scores, ld, n_c, rows, topk, cap, h1, idx, cnt);
+  k_topk<<<grid, kTopkThreads, smem, s>>>(scores, ld, n_c, rows, topk, cap, idx, cnt);
   QSA_CHECK_LAUNCH();
   return QSA_OK;
 }
@@ -335,10 +323,15 @@ qsa_status check_prefill_ptrs(std::initializer_list<const void*> ptrs) {
 // ---- decode geometry --------------------------------------------------------------------
 struct DecodeGeom {
   int32_t B = 0, cap = 0, topk = 512, max_nc = 0, splits = 4;
+  int32_t cand_cap = 0;   // top-k candidates kept per row (finish kernel's shared memory)
   int64_t ld = 4;
   PlanLayout pl;
   size_t o_scores = 0, o_nc = 0, o_idx = 0, o_cnt = 0, o_plan = 0, o_po = 0, o_pm = 0, o_pl = 0,
-         o_hist = 0, total = 0;
+         o_hist = 0, o_ccnt = 0, o_cand = 0, total = 0;
+  // shared memory of k_topk_finish
+  int finish_smem() const {
+    return kTopkSharedBytes + cand_cap * 8 + 2 * ((std::max(max_nc, 1) + 31) / 32) * 4;
+  }
 };
 
 qsa_status decode_geom(const qsa_cache* c, const qsa_params& p, DecodeGeom* g) {
@@ -365,7 +358,11 @@ qsa_status decode_geom(const qsa_cache* c, const qsa_params& p, DecodeGeom* g) {
   g->o_po = cv.take(parts * kHeadDim * 4);
   g->o_pm = cv.take(parts * 4);
   g->o_pl = cv.take(parts * 4);
-  g->o_hist = cv.take(static_cast<size_t>(g->B) * kTopkBins * 4);
+  // histograms and candidate counters sit back to back: one memset clears both
+  g->o_hist = cv.take(static_cast<size_t>(g->B) * kTopkBins * 4 + static_cast<size_t>(g->B) * 4);
+  g->o_ccnt = g->o_hist + static_cast<size_t>(g->B) * kTopkBins * 4;
+  g->cand_cap = std::min(kCandCap, static_cast<int>(round_up(std::max(g->max_nc, 64), 64)));
+  g->o_cand = cv.take(static_cast<size_t>(g->B) * g->cand_cap * 8);
   g->total = cv.off;
   return QSA_OK;
 }
@@ -674,9 +671,14 @@ qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, 
   int32_t* idx = sel_idx ? sel_idx : reinterpret_cast<int32_t*>(ws + g.o_idx);
   int32_t* cnt = sel_cnt ? sel_cnt : reinterpret_cast<int32_t*>(ws + g.o_cnt);
   int32_t* plan = reinterpret_cast<int32_t*>(ws + g.o_plan);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(ws + g.o_hist);
+  int32_t* cand_cnt = reinterpret_cast<int32_t*>(ws + g.o_ccnt);
+  uint64_t* cand = reinterpret_cast<uint64_t*>(ws + g.o_cand);
   const int sms = num_sms();
   const int max_nc_now = (max_len - 1) / 4;
-  // a2: scores (one token x 16 heads per sequence, split over M-tiles)
+  if (cudaMemsetAsync(hist, 0, static_cast<size_t>(g.B) * (kTopkBins + 1) * 4, s) != cudaSuccess)
+    return QSA_ERR_CUDA;
+  // a2: scores, with the first radix digit's histogram of every row (one token x 16 heads per sequence, split over M-tiles)
   {
     CUtensorMap tm_kbar, tm_qidx;
     const uint64_t dk[2] = {64, static_cast<uint64_t>(g.B) * (g.cap / 4)};
@@ -699,6 +701,7 @@ qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, 
     a.mtiles_per_split = per;
     a.kbar_rows_per_seq = g.cap / 4;
     a.n_c_out = n_c;
+    a.hist = hist;
     a.w = reinterpret_cast<const __nv_bfloat16*>(w);
     a.scores = scores;
     a.ld = g.ld;
@@ -706,10 +709,19 @@ qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, 
     k_index_score<1><<<g.B * splits, C::kThreads, C::kSmemBytes, s>>>(tm_kbar, tm_qidx, a);
     QSA_CHECK_LAUNCH();
   }
-  // a3: top-k
-  st = launch_topk(scores, g.ld, n_c, g.B, g.topk, max_nc_now, idx, cnt, s,
-                   reinterpret_cast<uint32_t*>(ws + g.o_hist));
-  if (st != QSA_OK) return st;
+  // a3: top-k: candidates at or above the threshold bin, then the exact select per row
+  {
+    const int parts = std::max(1, std::min((4 * sms + g.B - 1) / g.B, (max_nc_now + 2047) / 2048));
+    k_topk_collect<<<g.B * parts, kCandThreads, 0, s>>>(scores, g.ld, n_c, g.topk, parts,
+                                                         g.cand_cap, hist, cand_cnt, cand);
+    QSA_CHECK_LAUNCH();
+    const int smem = g.finish_smem();
+    if (!set_smem(k_topk_finish, smem)) return QSA_ERR_CUDA;
+    k_topk_finish<<<g.B, kTopkThreads, smem, s>>>(scores, g.ld, n_c, g.topk, g.cand_cap,
+                                                   std::max(g.max_nc, 1), hist, cand_cnt, cand,
+                                                   idx, cnt);
+    QSA_CHECK_LAUNCH();
+  }
   // union plan (one token per tile)
   {
     const int max_words = (g.cap - 1) / 4 / 32 + 1;

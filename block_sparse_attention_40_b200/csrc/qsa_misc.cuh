@@ -326,9 +326,8 @@ __global__ void k_append_len(int32_t* len, const int32_t* counts, int32_t n_new,
 // Step a3: top-k per row by radix select on order-preserving uint32 keys, digits of 12, 12
 // and 8 bits, then an ordered compaction that emits the selected blocks in ascending index
 // order and breaks ties at the threshold toward lower indices.  One 512-thread CTA per row;
-// a row of at most `smem_cap` scores is first copied to shared memory.  When `hist1` is
-// given (long decode rows), the first-digit histogram was built by k_topk_hist across many
-// CTAs and is read from there.
+// a row of at most `smem_cap` scores is first copied to shared memory.  topk_row takes the
+// first-digit histogram ready-made when one is given (decode rows, built while scoring).
 constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kTopkBins = 4096;
@@ -470,7 +469,6 @@ __device__ __forceinline__ void topk_row(const float* __restrict__ src, int n, i
 __global__ void __launch_bounds__(kTopkThreads) k_topk(const float* __restrict__ scores, int64_t ld,
                                                        const int32_t* __restrict__ n_c, int64_t rows,
                                                        int topk, int smem_cap,
-                                                       const uint32_t* __restrict__ hist1,
                                                        int32_t* __restrict__ idx,
                                                        int32_t* __restrict__ cnt) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -494,40 +492,187 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float* __restrict__
       src = row_cache;
       __syncthreads();
     }
-    topk_row(src, n, topk, hist1 ? hist1 + r * kTopkBins : nullptr, out, S);
+    topk_row(src, n, topk, nullptr, out, S);
     if (tid == 0) cnt[r] = topk;
   }
 }
 
-// First-digit histograms of long rows, split over `parts` CTAs per row (global atomics into
-// hist [rows][4096], which the caller zeroes).  Rows with n_c <= topk are skipped.
-__global__ void __launch_bounds__(kTopkThreads) k_topk_hist(const float* __restrict__ scores,
-                                                            int64_t ld, const int32_t* __restrict__ n_c,
-                                                            int topk, int parts,
-                                                            uint32_t* __restrict__ hist) {
-  __shared__ uint32_t h[kTopkBins];
+// ---------------------------------------------------------------------------------------
+// Long rows (decode): top-k from a first-digit histogram built while scoring, in two steps.
+//   k_topk_collect  (rows x parts CTAs): every CTA finds the threshold bin B1 of its row from
+//                   the histogram and appends (key, index) of each score in bins >= B1 to the
+//                   row's candidate list (at most topk - 1 + hist[B1] entries).
+//   k_topk_finish   (one CTA per row): exact radix select among the candidates (digits 2, 3),
+//                   then the ascending index list through shared-memory bitmaps: every key
+//                   above the threshold, plus the lowest-index keys equal to it.
+// A row whose candidates would not fit `cap` is left to the full-row path (k_topk).
+constexpr int kCandThreads = 256;
+
+__device__ __forceinline__ int hist_threshold_bin(const uint32_t* h, int topk, int* above_out,
+                                                  int* sh /*[40]*/) {
+  // bins scanned from the top; kCandThreads threads x 16 bins
+  const int tid = threadIdx.x;
+  const int per = 4096 / kCandThreads;
+  const int hi = 4095 - tid * per;
+  int local = 0;
+  for (int b = hi; b > hi - per; --b) local += static_cast<int>(h[b]);
+  int tot;
+  const int ex = block_excl_scan(local, sh, &tot);
+  int running = ex;
+  for (int b = hi; b > hi - per; --b) {
+    const int c = static_cast<int>(h[b]);
+    if (running < topk && running + c >= topk) {
+      sh[36] = b;
+      sh[37] = running;
+    }
+    running += c;
+  }
+  __syncthreads();
+  const int bin = sh[36];
+  *above_out = sh[37];
+  __syncthreads();
+  return bin;
+}
+
+__global__ void __launch_bounds__(kCandThreads) k_topk_collect(
+    const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_c, int topk,
+    int parts, int cap, const uint32_t* __restrict__ hist, int32_t* __restrict__ cand_cnt,
+    uint64_t* __restrict__ cand) {
+  __shared__ int sh[40];
   const int r = blockIdx.x / parts, part = blockIdx.x % parts;
   const int n = n_c[r];
   if (n <= topk) return;
-  const int lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i < kTopkBins; i += blockDim.x) h[i] = 0;
-  __syncthreads();
+  const uint32_t* h = hist + static_cast<int64_t>(r) * 4096;
+  int above;
+  const uint32_t b1 = static_cast<uint32_t>(hist_threshold_bin(h, topk, &above, sh));
+  if (above + static_cast<int>(h[b1]) > cap) return;   // overflow: full-row path later
   const int per = (n + parts - 1) / parts;
-  const int a = part * per, b = min(n, a + per);
+  const int a = part * per, e = min(n, a + per);
   const float* src = scores + static_cast<int64_t>(r) * ld;
-  for (int base = a; base < b; base += kTopkThreads) {
+  int32_t* cnt = cand_cnt + r;
+  uint64_t* out = cand + static_cast<int64_t>(r) * cap;
+  const int lane = threadIdx.x & 31;
+  for (int base = a; base < e; base += kCandThreads) {
     const int i = base + threadIdx.x;
-    const uint32_t bin = i < b ? (float_key(src[i]) >> 20) : 0xffffffffu;
-    const unsigned act = __ballot_sync(0xffffffffu, i < b);
-    if (i < b) {
-      const unsigned peers = __match_any_sync(act, bin);
-      if (lane == __ffs(peers) - 1) atomicAdd(&h[bin], static_cast<uint32_t>(__popc(peers)));
+    const uint32_t key = i < e ? float_key(src[i]) : 0u;
+    const bool take = i < e && (key >> 20) >= b1;
+    const unsigned m = __ballot_sync(0xffffffffu, take);
+    if (m == 0) continue;
+    int slot0 = 0;
+    if (lane == 0) slot0 = atomicAdd(cnt, __popc(m));
+    slot0 = __shfl_sync(0xffffffffu, slot0, 0);
+    if (take) {
+      const int slot = slot0 + __popc(m & ((1u << lane) - 1u));
+      if (slot < cap) out[slot] = (static_cast<uint64_t>(key) << 32) | static_cast<uint32_t>(i);
+    }
+  }
+}
+
+// Shared memory: TopkShared, then cap candidates (uint64), then two bitmaps of n_max bits.
+__global__ void __launch_bounds__(kTopkThreads) k_topk_finish(
+    const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_c, int topk,
+    int cap, int n_max, const uint32_t* __restrict__ hist, const int32_t* __restrict__ cand_cnt,
+    const uint64_t* __restrict__ cand, int32_t* __restrict__ idx, int32_t* __restrict__ cnt) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  TopkShared& S = *reinterpret_cast<TopkShared*>(smem_raw);
+  uint64_t* c = reinterpret_cast<uint64_t*>(smem_raw + kTopkSharedBytes);
+  const int nwords = (n_max + 31) / 32;
+  uint32_t* sel = reinterpret_cast<uint32_t*>(c + cap);
+  uint32_t* eqb = sel + nwords;
+  const int tid = threadIdx.x;
+  const int r = blockIdx.x;
+  const int n = n_c[r];
+  int32_t* out = idx + static_cast<int64_t>(r) * topk;
+  if (n <= topk) {
+    for (int i = tid; i < topk; i += blockDim.x) out[i] = i < n ? i : -1;
+    if (tid == 0) cnt[r] = n < 0 ? 0 : n;
+    return;
+  }
+  const uint32_t* h = hist + static_cast<int64_t>(r) * 4096;
+  for (int i = tid; i < kTopkBins; i += blockDim.x) S.hist[i] = h[i];
+  __syncthreads();
+  int need = topk, above;
+  const uint32_t b1 = static_cast<uint32_t>(topk_find_bin(S, kTopkBins, need, &above));
+  need -= above;
+  const int C = cand_cnt[r];
+  const int in_b1 = static_cast<int>(S.hist[b1]);
+  __syncthreads();   // every thread has read the histogram before it is cleared below
+  if (above + in_b1 > cap || C > cap) {
+    // the candidates did not fit: full-row radix select on the scores in global memory
+    topk_row(scores + static_cast<int64_t>(r) * ld, n, topk, h, out, S);
+    if (tid == 0) cnt[r] = topk;
+    return;
+  }
+  for (int i = tid; i < C; i += blockDim.x) c[i] = cand[static_cast<int64_t>(r) * cap + i];
+  for (int i = tid; i < kTopkBins; i += blockDim.x) S.hist[i] = 0;
+  for (int i = tid; i < 2 * nwords; i += blockDim.x) sel[i] = 0;   // sel and eqb
+  __syncthreads();
+  // digit 2 among candidates in bin b1
+  for (int i = tid; i < C; i += blockDim.x) {
+    const uint32_t key = static_cast<uint32_t>(c[i] >> 32);
+    if ((key >> 20) == b1) atomicAdd(&S.hist[(key >> 8) & 0xfffu], 1u);
+  }
+  __syncthreads();
+  const uint32_t b2 = static_cast<uint32_t>(topk_find_bin(S, kTopkBins, need, &above));
+  need -= above;
+  const uint32_t pre = (b1 << 12) | b2;
+  for (int i = tid; i < 256; i += blockDim.x) S.hist[i] = 0;
+  __syncthreads();
+  for (int i = tid; i < C; i += blockDim.x) {
+    const uint32_t key = static_cast<uint32_t>(c[i] >> 32);
+    if ((key >> 8) == pre) atomicAdd(&S.hist[key & 0xffu], 1u);
+  }
+  __syncthreads();
+  const uint32_t b3 = static_cast<uint32_t>(topk_find_bin(S, 256, need, &above));
+  need -= above;
+  const uint32_t T = (pre << 8) | b3;
+  const int need_eq = need;
+  // bitmaps: keys above T are selected; keys equal to T are marked in eqb
+  for (int i = tid; i < C; i += blockDim.x) {
+    const uint32_t key = static_cast<uint32_t>(c[i] >> 32);
+    const uint32_t ix = static_cast<uint32_t>(c[i]);
+    if (key > T) atomicOr(&sel[ix >> 5], 1u << (ix & 31));
+    else if (key == T) atomicOr(&eqb[ix >> 5], 1u << (ix & 31));
+  }
+  __syncthreads();
+  // the need_eq lowest equal keys join the selection: prefix popcounts over eqb
+  {
+    const int per = (nwords + kTopkThreads - 1) / kTopkThreads;
+    const int w0 = tid * per;
+    int local = 0;
+    for (int w = w0; w < min(nwords, w0 + per); ++w) local += __popc(eqb[w]);
+    int tot;
+    int before = block_excl_scan(local, S.sh, &tot);
+    for (int w = w0; w < min(nwords, w0 + per); ++w) {
+      uint32_t bits = eqb[w];
+      while (bits && before < need_eq) {
+        const uint32_t low = bits & (0u - bits);
+        sel[w] |= low;
+        bits ^= low;
+        ++before;
+      }
     }
   }
   __syncthreads();
-  uint32_t* dst = hist + static_cast<int64_t>(r) * kTopkBins;
-  for (int i = threadIdx.x; i < kTopkBins; i += blockDim.x)
-    if (h[i]) atomicAdd(&dst[i], h[i]);
+  // ascending output: prefix popcounts over sel
+  {
+    const int per = (nwords + kTopkThreads - 1) / kTopkThreads;
+    const int w0 = tid * per;
+    int local = 0;
+    for (int w = w0; w < min(nwords, w0 + per); ++w) local += __popc(sel[w]);
+    int tot;
+    int pos = block_excl_scan(local, S.sh, &tot);
+    for (int w = w0; w < min(nwords, w0 + per); ++w) {
+      uint32_t bits = sel[w];
+      while (bits) {
+        const int b = __ffs(bits) - 1;
+        bits &= bits - 1;
+        if (pos < topk) out[pos] = w * 32 + b;
+        ++pos;
+      }
+    }
+  }
+  if (tid == 0) cnt[r] = topk;
 }
 
 // ---------------------------------------------------------------------------------------

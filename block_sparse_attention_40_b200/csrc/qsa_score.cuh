@@ -34,7 +34,10 @@ struct ScoreCfg {
   static constexpr int kWOff = kBOff + ((kBBytes + 1023) / 1024) * 1024;
   static constexpr int kBarOff = kWOff + NTOK * kIdxHeads * 4;
   static constexpr int kNumBars = 2 * kStages + 2 * kNumAcc + 2;
-  static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;  // + align slack
+  // decode: first-digit (key bits 31..20) histogram of this CTA's scores, flushed to global
+  static constexpr int kHistOff = kBarOff + kNumBars * 8 + 16;
+  static constexpr int kHistBytes = NTOK == 1 ? 4096 * 4 : 0;
+  static constexpr int kSmemBytes = kHistOff + kHistBytes + 1024;  // + align slack
   static constexpr uint32_t kIdesc = idesc_bf16_f32(128, kN, 0, 0);
 };
 
@@ -52,6 +55,7 @@ struct ScoreArgs {
   int32_t mtiles_per_split;
   int64_t kbar_rows_per_seq;
   int32_t* n_c_out;        // [B] n_c per sequence (written by split 0), may be null
+  uint32_t* hist;          // [B][4096] first-digit histograms of the scores (zeroed), or null
   // common
   const __nv_bfloat16* w;  // prefill: [T][16]; decode: [B][16]
   float* scores;
@@ -149,6 +153,10 @@ __global__ void __launch_bounds__(ScoreCfg<NTOK>::kThreads, 1)
     mbar_init(mma_done, 1);
     *s_abort = 0;
     fence_mbar_init();
+  }
+  uint32_t* sHist = reinterpret_cast<uint32_t*>(smem + C::kHistOff);
+  if constexpr (NTOK == 1) {
+    for (int i = threadIdx.x; i < 4096; i += blockDim.x) sHist[i] = 0;
   }
   // weights of the tile's tokens, widened to fp32
   for (int i = threadIdx.x; i < NTOK * kIdxHeads; i += blockDim.x) {
@@ -252,12 +260,29 @@ __global__ void __launch_bounds__(ScoreCfg<NTOK>::kThreads, 1)
           s = fmaf(sW[tok * kIdxHeads + h], fmaxf(x, 0.f), s);
         }
         const int pos = wk.pos0 + tok;
-        if (tok < wk.ntok && blk < pos / kBlock)
-          args.scores[(wk.out_row0 + tok) * args.ld + blk] = s;
+        const bool valid = tok < wk.ntok && blk < pos / kBlock;
+        if (valid) args.scores[(wk.out_row0 + tok) * args.ld + blk] = s;
+        if constexpr (NTOK == 1) {
+          if (args.hist) {
+            const unsigned act = __ballot_sync(0xffffffffu, valid);
+            if (valid) {
+              const uint32_t bin = float_key(s) >> 20;
+              const unsigned peers = __match_any_sync(act, bin);
+              if (lane == __ffs(peers) - 1) atomicAdd(&sHist[bin], static_cast<uint32_t>(__popc(peers)));
+            }
+          }
+        }
       }
     }
   }
   __syncthreads();
+  if constexpr (NTOK == 1) {
+    if (args.hist) {
+      uint32_t* dst = args.hist + static_cast<int64_t>(wk.out_row0) * 4096;
+      for (int i = threadIdx.x; i < 4096; i += blockDim.x)
+        if (sHist[i]) atomicAdd(&dst[i], sHist[i]);
+    }
+  }
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();

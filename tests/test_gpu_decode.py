@@ -32,9 +32,14 @@ def _oracle_row(k_tok, v_tok, kidx_tok, q, q_idx, w, topk, forced=None):
     return idx, cnt, kth, out, kbar
 
 
-def _decode_session(spec, check_seqs, steps, splits=0, device_gen=False):
+def _decode_session(spec, check_seqs, steps, splits=0, device_gen=False, ctx_fn=None,
+                    step_fn=None, exact_sel=False):
+    """ctx_fn(k, v, k_idx) and step_fn(step dict) may reshape the seeded inputs (ties);
+    exact_sel demands the oracle's selection itself (inputs whose scores are exact)."""
     gen_dev = DEV if device_gen else "cpu"
     k_ctx, v_ctx, ki_ctx = W.decode_context(spec, device=gen_dev)
+    if ctx_fn is not None:
+        k_ctx, v_ctx, ki_ctx = ctx_fn(k_ctx, v_ctx, ki_ctx)
     cache = qsa.KVCache(spec.batch, spec.capacity, DEV, zero=False)
     # bulk fill in chunks with per-sequence counts
     lmax = max(spec.context)
@@ -52,6 +57,8 @@ def _decode_session(spec, check_seqs, steps, splits=0, device_gen=False):
     results = []
     for step in range(steps):
         st = W.decode_step(spec, step, device=gen_dev)
+        if step_fn is not None:
+            st = step_fn(st)
         cache.append(st["k"].to(DEV), st["v"].to(DEV), st["k_idx"].to(DEV))
         out, idx, cnt = dec.run(st["q"].to(DEV), st["q_idx"].to(DEV), st["w"].to(DEV),
                                 with_selection=True)
@@ -73,7 +80,8 @@ def _decode_session(spec, check_seqs, steps, splits=0, device_gen=False):
                                           np.array([0, L]), np.zeros(1, np.int64),
                                           np.zeros(len(blocks), np.int64), blocks)
 
-            swaps = compare_selection(g_idx, g_cnt, o_idx, o_cnt, o_kth, score_fn)
+            swaps = compare_selection(g_idx, g_cnt, o_idx, o_cnt, o_kth, score_fn,
+                                      exact=exact_sel)
             _, _, _, o_out, _ = _oracle_row(kt, vt, kit, q, qi, w, spec.topk,
                                             forced=(g_idx, g_cnt))
             results.append((b, step, swaps) + compare_outputs(out[b:b + 1], o_out))
@@ -102,6 +110,49 @@ def test_decode_short_contexts():
     spec = W.small_decode_spec(batch=4, context=(0, 1, 3, 6), capacity=64, topk=512, steps=5,
                                seed=9)
     _decode_session(spec, check_seqs=[0, 1, 2, 3], steps=5)
+
+
+def _int_ctx(k, v, ki):
+    return k, v, torch.round(ki.float()).clamp(-3, 3).to(torch.bfloat16)
+
+
+def _int_step(st):
+    st = dict(st)
+    st["k_idx"] = torch.round(st["k_idx"].float()).clamp(-3, 3).to(torch.bfloat16)
+    st["q_idx"] = torch.round(st["q_idx"].float()).clamp(-3, 3).to(torch.bfloat16)
+    st["w"] = torch.round(st["w"].float()).to(torch.bfloat16)
+    return st
+
+
+def _zero_w(st):
+    st = dict(st)
+    st["w"] = torch.zeros_like(st["w"])
+    return st
+
+
+def test_decode_integer_scores_ties():
+    # small-integer indexer inputs: scores are exact multiples of 1/4 with many equal values
+    # at the threshold, which the selection breaks toward lower block indices
+    spec = W.small_decode_spec(batch=3, context=(5001, 5002, 6003), capacity=6100, topk=96,
+                               steps=3, seed=21)
+    _decode_session(spec, check_seqs=[0, 1, 2], steps=3, ctx_fn=_int_ctx, step_fn=_int_step,
+                    exact_sel=True)
+
+
+def test_decode_all_scores_equal():
+    # w = 0: every score is 0, so the selection is the lowest topk block indices
+    spec = W.small_decode_spec(batch=2, context=(4000, 4097), capacity=4200, topk=64, steps=2,
+                               seed=22)
+    res = _decode_session(spec, check_seqs=[0, 1], steps=2, step_fn=_zero_w, exact_sel=True)
+    assert len(res) == 4
+
+
+def test_decode_candidate_overflow_all_equal():
+    # w = 0 on rows of more than 16384 complete blocks: the threshold bin holds every block,
+    # more than the candidate buffer, so the rows take the full-row select
+    spec = W.small_decode_spec(batch=2, context=(70001, 73000), capacity=73100, topk=512,
+                               steps=1, seed=23)
+    _decode_session(spec, check_seqs=[0, 1], steps=1, step_fn=_zero_w, exact_sel=True)
 
 
 @pytest.mark.slow
