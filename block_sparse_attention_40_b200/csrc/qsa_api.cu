@@ -21,7 +21,7 @@ namespace {
 constexpr int kVersion = 100;   // 0.1.0
 constexpr int kDefaultRowsPerTile = 10;
 constexpr int kDefaultScoreChunkRows = 16384;
-constexpr int kTopkSmemCap = 32768;     // row scores cached in shared memory up to this n_c
+constexpr int kTopkCandCap = 4096;      // per-row candidates of the score-row top-k
 constexpr int kCandCap = 16384;         // decode top-k candidates per row
 constexpr int kNumSMsFallback = 148;
 
@@ -191,15 +191,16 @@ qsa_status launch_compress(const void* k_idx, const SeqMeta* meta, int num_seqs,
   return QSA_OK;
 }
 
-// Top-k over `rows` score rows (one CTA per row; short rows cached in shared memory).
+// Top-k over `rows` score rows (one CTA per row, grid-strided).
 qsa_status launch_topk(const float* scores, int64_t ld, const int32_t* n_c, int64_t rows,
                        int topk, int max_nc, int32_t* idx, int32_t* cnt, cudaStream_t s) {
   if (rows <= 0) return QSA_OK;
-  const int cap = std::min(max_nc, kTopkSmemCap);
-  const int smem = kTopkSharedBytes + std::max(cap, 0) * 4;
+  const int n_max = std::max(max_nc, 1);
+  const int smem = kTopkSharedBytes + kTopkCandCap * 8 + 2 * ((n_max + 31) / 32) * 4;
   if (!set_smem(k_topk, smem)) return QSA_ERR_CUDA;
-  const int grid = static_cast<int>(std::min<int64_t>(rows, int64_t(num_sms()) * 8));
-  k_topk<<<grid, kTopkThreads, smem, s>>>(scores, ld, n_c, rows, topk, cap, idx, cnt);
+  const int grid = static_cast<int>(std::min<int64_t>(rows, int64_t(num_sms()) * 16));
+  k_topk<<<grid, kTopkThreads, smem, s>>>(scores, ld, n_c, rows, topk, kTopkCandCap, n_max, idx,
+                                          cnt);
   QSA_CHECK_LAUNCH();
   return QSA_OK;
 }
@@ -233,12 +234,12 @@ qsa_status run_scores_and_topk(const void* q_idx, const void* w, const void* kba
     const uint32_t box[2] = {64, 256};
     if (!make_tmap(&tm_qidx, q_idx, 2, dims, strides, box)) return QSA_ERR_CUDA;
   }
-  using C = ScoreCfg<16>;
-  const int smem = std::max(C::kSmemBytes, 116 * 1024);   // one CTA per SM (512 TMEM columns)
-  if (!set_smem(k_index_score<16>, smem)) return QSA_ERR_CUDA;
   std::vector<int64_t> starts;
   score_tile_token_starts(h_cu, num_seqs, &starts);
   const int ntiles = static_cast<int>(starts.size()) - 1;
+  using C = ScoreCfg<16>;
+  const int smem = std::max(C::kSmemBytes, 116 * 1024);   // one CTA per SM (512 TMEM columns)
+  if (!set_smem(k_index_score<16>, smem)) return QSA_ERR_CUDA;
   int t = 0;
   while (t < ntiles) {
     int e = t + 1;
@@ -711,7 +712,8 @@ qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, 
   }
   // a3: top-k: candidates at or above the threshold bin, then the exact select per row
   {
-    const int parts = std::max(1, std::min((4 * sms + g.B - 1) / g.B, (max_nc_now + 2047) / 2048));
+    // one pass of 4096 scores per CTA
+    const int parts = std::max(1, (max_nc_now + 4095) / 4096);
     k_topk_collect<<<g.B * parts, kCandThreads, 0, s>>>(scores, g.ld, n_c, g.topk, parts,
                                                          g.cand_cap, hist, cand_cnt, cand);
     QSA_CHECK_LAUNCH();

@@ -16,6 +16,19 @@ struct SeqMeta {
   int32_t pad;
 };
 
+// Warp-wide exclusive scan of one int per lane; *total receives the warp sum.
+__device__ __forceinline__ int warp_count_scan(int v, int* total) {
+  const int lane = threadIdx.x & 31;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  *total = __shfl_sync(0xffffffffu, x, 31);
+  return x - v;
+}
+
 // ---------------------------------------------------------------------------------------
 // Block-wide exclusive scan of one int per thread (blockDim.x a multiple of 32, <= 1024).
 __device__ __forceinline__ int block_excl_scan(int v, int* sh /*[33]*/, int* total) {
@@ -323,11 +336,13 @@ __global__ void k_append_len(int32_t* len, const int32_t* counts, int32_t n_new,
 }
 
 // ---------------------------------------------------------------------------------------
-// Step a3: top-k per row by radix select on order-preserving uint32 keys, digits of 12, 12
-// and 8 bits, then an ordered compaction that emits the selected blocks in ascending index
-// order and breaks ties at the threshold toward lower indices.  One 512-thread CTA per row;
-// a row of at most `smem_cap` scores is first copied to shared memory.  topk_row takes the
-// first-digit histogram ready-made when one is given (decode rows, built while scoring).
+// Step a3: top-k per row by radix select on order-preserving uint32 keys, with the selected
+// blocks emitted in ascending index order and ties at the threshold broken toward lower
+// indices.  One 512-thread CTA works on a row.  The kernels (k_topk for score rows; the
+// collect/finish pair for decode) narrow a row to the candidates at or above the threshold bin
+// of the first digit (key bits 31..20) and finish there; topk_row, the full-row select with
+// digits of 12, 12 and 8 bits and an ordered compaction over the whole row, serves rows whose
+// candidates overflow.  It takes the first-digit histogram ready-made when one is given.
 constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kTopkBins = 4096;
@@ -466,36 +481,6 @@ __device__ __forceinline__ void topk_row(const float* __restrict__ src, int n, i
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(kTopkThreads) k_topk(const float* __restrict__ scores, int64_t ld,
-                                                       const int32_t* __restrict__ n_c, int64_t rows,
-                                                       int topk, int smem_cap,
-                                                       int32_t* __restrict__ idx,
-                                                       int32_t* __restrict__ cnt) {
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  TopkShared& S = *reinterpret_cast<TopkShared*>(smem_raw);
-  float* row_cache = reinterpret_cast<float*>(smem_raw + kTopkSharedBytes);
-  const int tid = threadIdx.x;
-  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
-    const int n = n_c[r];
-    int32_t* out = idx + r * topk;
-    if (n <= topk) {
-      for (int i = tid; i < topk; i += blockDim.x) out[i] = i < n ? i : -1;
-      if (tid == 0) cnt[r] = n < 0 ? 0 : n;
-      continue;
-    }
-    const float* src = scores + r * ld;
-    if (n <= smem_cap) {
-      const int n4 = n >> 2;
-      const float4* s4 = reinterpret_cast<const float4*>(src);
-      for (int i = tid; i < n4; i += blockDim.x) reinterpret_cast<float4*>(row_cache)[i] = s4[i];
-      for (int i = 4 * n4 + tid; i < n; i += blockDim.x) row_cache[i] = src[i];
-      src = row_cache;
-      __syncthreads();
-    }
-    topk_row(src, n, topk, nullptr, out, S);
-    if (tid == 0) cnt[r] = topk;
-  }
-}
 
 // ---------------------------------------------------------------------------------------
 // Long rows (decode): top-k from a first-digit histogram built while scoring, in two steps.
@@ -505,109 +490,125 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float* __restrict__
 //   k_topk_finish   (one CTA per row): exact radix select among the candidates (digits 2, 3),
 //                   then the ascending index list through shared-memory bitmaps: every key
 //                   above the threshold, plus the lowest-index keys equal to it.
-// A row whose candidates would not fit `cap` is left to the full-row path (k_topk).
+// A row whose candidates would not fit `cap` is left to the full-row select (topk_row).
 constexpr int kCandThreads = 256;
+static_assert(kCandThreads * 16 == 4096, "hist_threshold_bin gives each thread 16 bins");
 
-__device__ __forceinline__ int hist_threshold_bin(const uint32_t* h, int topk, int* above_out,
-                                                  int* sh /*[40]*/) {
-  // bins scanned from the top; kCandThreads threads x 16 bins
-  const int tid = threadIdx.x;
-  const int per = 4096 / kCandThreads;
-  const int hi = 4095 - tid * per;
+// Threshold bin of a row from its 4096-bin histogram: thread t holds bins 4080-16t .. 4095-16t
+// in registers (the highest bins go to thread 0).  Returns the bin where the count of keys in
+// higher bins first reaches `topk`; *above receives that count and *in_bin the bin's own.
+__device__ __forceinline__ int hist_threshold_bin(const uint32_t* __restrict__ h, int topk,
+                                                  int* above_out, int* in_bin_out, int* sh /*[40]*/) {
+  const int lo = 4080 - 16 * static_cast<int>(threadIdx.x);
+  const uint4* h4 = reinterpret_cast<const uint4*>(h + lo);
+  uint32_t v[16];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 x = h4[q];
+    v[4 * q] = x.x;
+    v[4 * q + 1] = x.y;
+    v[4 * q + 2] = x.z;
+    v[4 * q + 3] = x.w;
+  }
   int local = 0;
-  for (int b = hi; b > hi - per; --b) local += static_cast<int>(h[b]);
+#pragma unroll
+  for (int j = 0; j < 16; ++j) local += static_cast<int>(v[j]);
   int tot;
-  const int ex = block_excl_scan(local, sh, &tot);
-  int running = ex;
-  for (int b = hi; b > hi - per; --b) {
-    const int c = static_cast<int>(h[b]);
+  int running = block_excl_scan(local, sh, &tot);   // keys in bins above this thread's range
+#pragma unroll
+  for (int j = 15; j >= 0; --j) {
+    const int c = static_cast<int>(v[j]);
     if (running < topk && running + c >= topk) {
-      sh[36] = b;
+      sh[36] = lo + j;
       sh[37] = running;
+      sh[38] = c;
     }
     running += c;
   }
   __syncthreads();
   const int bin = sh[36];
   *above_out = sh[37];
+  *in_bin_out = sh[38];
   __syncthreads();
   return bin;
 }
 
+// Each CTA covers `per` (a multiple of 4) scores of one row in passes of 16 scores a thread:
+// all loads of a pass are issued before one block scan places the pass's candidates, so a
+// pass costs one load latency and one atomic on the row's counter.
+constexpr int kCollectPerThread = 16;
 __global__ void __launch_bounds__(kCandThreads) k_topk_collect(
     const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_c, int topk,
     int parts, int cap, const uint32_t* __restrict__ hist, int32_t* __restrict__ cand_cnt,
     uint64_t* __restrict__ cand) {
   __shared__ int sh[40];
+  __shared__ int s_base;
   const int r = blockIdx.x / parts, part = blockIdx.x % parts;
   const int n = n_c[r];
   if (n <= topk) return;
-  const uint32_t* h = hist + static_cast<int64_t>(r) * 4096;
-  int above;
-  const uint32_t b1 = static_cast<uint32_t>(hist_threshold_bin(h, topk, &above, sh));
-  if (above + static_cast<int>(h[b1]) > cap) return;   // overflow: full-row path later
-  const int per = (n + parts - 1) / parts;
+  int above, in_b1;
+  const uint32_t b1 = static_cast<uint32_t>(
+      hist_threshold_bin(hist + static_cast<int64_t>(r) * 4096, topk, &above, &in_b1, sh));
+  if (above + in_b1 > cap) return;   // overflow: the finish kernel takes the full-row path
+  const int per = ((n + parts - 1) / parts + 3) & ~3;
   const int a = part * per, e = min(n, a + per);
   const float* src = scores + static_cast<int64_t>(r) * ld;
-  int32_t* cnt = cand_cnt + r;
   uint64_t* out = cand + static_cast<int64_t>(r) * cap;
-  const int lane = threadIdx.x & 31;
-  for (int base = a; base < e; base += kCandThreads) {
-    const int i = base + threadIdx.x;
-    const uint32_t key = i < e ? float_key(src[i]) : 0u;
-    const bool take = i < e && (key >> 20) >= b1;
-    const unsigned m = __ballot_sync(0xffffffffu, take);
-    if (m == 0) continue;
-    int slot0 = 0;
-    if (lane == 0) slot0 = atomicAdd(cnt, __popc(m));
-    slot0 = __shfl_sync(0xffffffffu, slot0, 0);
-    if (take) {
-      const int slot = slot0 + __popc(m & ((1u << lane) - 1u));
-      if (slot < cap) out[slot] = (static_cast<uint64_t>(key) << 32) | static_cast<uint32_t>(i);
+  constexpr int kPass = kCandThreads * kCollectPerThread;
+  for (int base = a; base < e; base += kPass) {
+    float x[kCollectPerThread];
+#pragma unroll
+    for (int q = 0; q < kCollectPerThread / 4; ++q) {
+      const int i = base + 4 * (q * kCandThreads + static_cast<int>(threadIdx.x));
+      float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i < e) f = *reinterpret_cast<const float4*>(src + i);   // i % 4 == 0, row 16B-aligned
+      x[4 * q] = f.x;
+      x[4 * q + 1] = f.y;
+      x[4 * q + 2] = f.z;
+      x[4 * q + 3] = f.w;
     }
+    uint32_t take = 0;
+#pragma unroll
+    for (int j = 0; j < kCollectPerThread; ++j) {
+      const int i = base + 4 * ((j / 4) * kCandThreads + static_cast<int>(threadIdx.x)) + (j & 3);
+      if (i < e && (float_key(x[j]) >> 20) >= b1) take |= 1u << j;
+    }
+    int tot;
+    const int ex = block_excl_scan(__popc(take), sh, &tot);
+    if (tot == 0) continue;   // uniform: tot is the block total
+    if (threadIdx.x == 0) s_base = atomicAdd(cand_cnt + r, tot);
+    __syncthreads();
+    int slot = s_base + ex;
+#pragma unroll
+    for (int j = 0; j < kCollectPerThread; ++j) {
+      if (take & (1u << j)) {
+        const int i = base + 4 * ((j / 4) * kCandThreads + static_cast<int>(threadIdx.x)) + (j & 3);
+        if (slot < cap) out[slot] = (static_cast<uint64_t>(float_key(x[j])) << 32) | static_cast<uint32_t>(i);
+        ++slot;
+      }
+    }
+    __syncthreads();   // s_base is rewritten by the next pass
   }
 }
 
-// Shared memory: TopkShared, then cap candidates (uint64), then two bitmaps of n_max bits.
-__global__ void __launch_bounds__(kTopkThreads) k_topk_finish(
-    const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_c, int topk,
-    int cap, int n_max, const uint32_t* __restrict__ hist, const int32_t* __restrict__ cand_cnt,
-    const uint64_t* __restrict__ cand, int32_t* __restrict__ idx, int32_t* __restrict__ cnt) {
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  TopkShared& S = *reinterpret_cast<TopkShared*>(smem_raw);
-  uint64_t* c = reinterpret_cast<uint64_t*>(smem_raw + kTopkSharedBytes);
-  const int nwords = (n_max + 31) / 32;
-  uint32_t* sel = reinterpret_cast<uint32_t*>(c + cap);
-  uint32_t* eqb = sel + nwords;
+// Exact top-k among candidates c[0 .. C) (composites key << 32 | block, in any order) that hold
+// every key at or above the threshold bin b1 of the first digit; `need` is topk minus the keys
+// in bins above b1.  Digits 2 (key bits 19..8) and 3 (bits 7..0) among the keys of bin b1 give
+// the k-th largest key T; the selection is every key above T plus the need_eq lowest-index keys
+// equal to T, emitted in ascending block order through two bitmaps of nwords words (sel, eqb)
+// and prefix popcounts.  Called by all kTopkThreads threads of the CTA.
+__device__ __forceinline__ void topk_select_candidates(TopkShared& S, const uint64_t* c, int C,
+                                                       uint32_t b1, int need, uint32_t* sel,
+                                                       uint32_t* eqb, int nwords, int topk,
+                                                       int32_t* __restrict__ out) {
   const int tid = threadIdx.x;
-  const int r = blockIdx.x;
-  const int n = n_c[r];
-  int32_t* out = idx + static_cast<int64_t>(r) * topk;
-  if (n <= topk) {
-    for (int i = tid; i < topk; i += blockDim.x) out[i] = i < n ? i : -1;
-    if (tid == 0) cnt[r] = n < 0 ? 0 : n;
-    return;
-  }
-  const uint32_t* h = hist + static_cast<int64_t>(r) * 4096;
-  for (int i = tid; i < kTopkBins; i += blockDim.x) S.hist[i] = h[i];
-  __syncthreads();
-  int need = topk, above;
-  const uint32_t b1 = static_cast<uint32_t>(topk_find_bin(S, kTopkBins, need, &above));
-  need -= above;
-  const int C = cand_cnt[r];
-  const int in_b1 = static_cast<int>(S.hist[b1]);
-  __syncthreads();   // every thread has read the histogram before it is cleared below
-  if (above + in_b1 > cap || C > cap) {
-    // the candidates did not fit: full-row radix select on the scores in global memory
-    topk_row(scores + static_cast<int64_t>(r) * ld, n, topk, h, out, S);
-    if (tid == 0) cnt[r] = topk;
-    return;
-  }
-  for (int i = tid; i < C; i += blockDim.x) c[i] = cand[static_cast<int64_t>(r) * cap + i];
+  int above;
   for (int i = tid; i < kTopkBins; i += blockDim.x) S.hist[i] = 0;
-  for (int i = tid; i < 2 * nwords; i += blockDim.x) sel[i] = 0;   // sel and eqb
+  for (int i = tid; i < nwords; i += blockDim.x) {
+    sel[i] = 0;
+    eqb[i] = 0;
+  }
   __syncthreads();
-  // digit 2 among candidates in bin b1
   for (int i = tid; i < C; i += blockDim.x) {
     const uint32_t key = static_cast<uint32_t>(c[i] >> 32);
     if ((key >> 20) == b1) atomicAdd(&S.hist[(key >> 8) & 0xfffu], 1u);
@@ -635,15 +636,15 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk_finish(
     else if (key == T) atomicOr(&eqb[ix >> 5], 1u << (ix & 31));
   }
   __syncthreads();
+  const int per = (nwords + kTopkThreads - 1) / kTopkThreads;
+  const int w0 = tid * per, w1 = min(nwords, w0 + per);
   // the need_eq lowest equal keys join the selection: prefix popcounts over eqb
   {
-    const int per = (nwords + kTopkThreads - 1) / kTopkThreads;
-    const int w0 = tid * per;
     int local = 0;
-    for (int w = w0; w < min(nwords, w0 + per); ++w) local += __popc(eqb[w]);
+    for (int w = w0; w < w1; ++w) local += __popc(eqb[w]);
     int tot;
     int before = block_excl_scan(local, S.sh, &tot);
-    for (int w = w0; w < min(nwords, w0 + per); ++w) {
+    for (int w = w0; w < w1; ++w) {
       uint32_t bits = eqb[w];
       while (bits && before < need_eq) {
         const uint32_t low = bits & (0u - bits);
@@ -656,13 +657,11 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk_finish(
   __syncthreads();
   // ascending output: prefix popcounts over sel
   {
-    const int per = (nwords + kTopkThreads - 1) / kTopkThreads;
-    const int w0 = tid * per;
     int local = 0;
-    for (int w = w0; w < min(nwords, w0 + per); ++w) local += __popc(sel[w]);
+    for (int w = w0; w < w1; ++w) local += __popc(sel[w]);
     int tot;
     int pos = block_excl_scan(local, S.sh, &tot);
-    for (int w = w0; w < min(nwords, w0 + per); ++w) {
+    for (int w = w0; w < w1; ++w) {
       uint32_t bits = sel[w];
       while (bits) {
         const int b = __ffs(bits) - 1;
@@ -672,7 +671,146 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk_finish(
       }
     }
   }
+  __syncthreads();   // S and the bitmaps are reused by the caller's next row
+}
+
+// Shared memory: TopkShared, then cap candidates (uint64), then two bitmaps of n_max bits.
+__global__ void __launch_bounds__(kTopkThreads) k_topk_finish(
+    const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_c, int topk,
+    int cap, int n_max, const uint32_t* __restrict__ hist, const int32_t* __restrict__ cand_cnt,
+    const uint64_t* __restrict__ cand, int32_t* __restrict__ idx, int32_t* __restrict__ cnt) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  TopkShared& S = *reinterpret_cast<TopkShared*>(smem_raw);
+  uint64_t* c = reinterpret_cast<uint64_t*>(smem_raw + kTopkSharedBytes);
+  const int nwords = (n_max + 31) / 32;
+  uint32_t* sel = reinterpret_cast<uint32_t*>(c + cap);
+  uint32_t* eqb = sel + nwords;
+  const int tid = threadIdx.x;
+  const int r = blockIdx.x;
+  const int n = n_c[r];
+  int32_t* out = idx + static_cast<int64_t>(r) * topk;
+  if (n <= topk) {
+    for (int i = tid; i < topk; i += blockDim.x) out[i] = i < n ? i : -1;
+    if (tid == 0) cnt[r] = n < 0 ? 0 : n;
+    return;
+  }
+  const uint32_t* h = hist + static_cast<int64_t>(r) * 4096;
+  for (int i = tid; i < kTopkBins; i += blockDim.x) S.hist[i] = h[i];
+  __syncthreads();
+  int above;
+  const uint32_t b1 = static_cast<uint32_t>(topk_find_bin(S, kTopkBins, topk, &above));
+  const int C = cand_cnt[r];
+  const int in_b1 = static_cast<int>(S.hist[b1]);
+  __syncthreads();   // every thread has read the histogram before it is rewritten
+  if (above + in_b1 > cap || C > cap) {
+    // the candidates did not fit: full-row radix select on the scores in global memory
+    topk_row(scores + static_cast<int64_t>(r) * ld, n, topk, h, out, S);
+    if (tid == 0) cnt[r] = topk;
+    return;
+  }
+  for (int i = tid; i < C; i += blockDim.x) c[i] = cand[static_cast<int64_t>(r) * cap + i];
+  topk_select_candidates(S, c, C, b1, topk - above, sel, eqb, (n + 31) / 32, topk, out);
   if (tid == 0) cnt[r] = topk;
+}
+
+// Step a3 on score rows, one CTA per row (grid-strided): pass 1 reads the row and builds the
+// first-digit histogram (key bits 31..20); pass 2 reads it again (from L2) and collects the
+// composites of the keys at or above the threshold bin b1 into shared memory; the exact select
+// and the ordered output then run on those candidates (topk_select_candidates).  A row whose
+// candidates would exceed `cap` takes the full-row select (topk_row).  Rows whose start is
+// 16-byte aligned (ld a multiple of 4) are read as float4.
+// Shared memory: TopkShared, then cap candidates (uint64), then two bitmaps of n_max bits.
+__global__ void __launch_bounds__(kTopkThreads, 4) k_topk(const float* __restrict__ scores, int64_t ld,
+                                                       const int32_t* __restrict__ n_c, int64_t rows,
+                                                       int topk, int cap, int n_max,
+                                                       int32_t* __restrict__ idx,
+                                                       int32_t* __restrict__ cnt) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  TopkShared& S = *reinterpret_cast<TopkShared*>(smem_raw);
+  uint64_t* c = reinterpret_cast<uint64_t*>(smem_raw + kTopkSharedBytes);
+  uint32_t* sel = reinterpret_cast<uint32_t*>(c + cap);
+  uint32_t* eqb = sel + (n_max + 31) / 32;
+  __shared__ int s_cc;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const bool vec = (ld & 3) == 0;
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const int n = n_c[r];
+    int32_t* out = idx + r * topk;
+    if (n <= topk) {
+      for (int i = tid; i < topk; i += blockDim.x) out[i] = i < n ? i : -1;
+      if (tid == 0) cnt[r] = n < 0 ? 0 : n;
+      continue;
+    }
+    const float* src = scores + r * ld;
+    // ---- pass 1: first-digit histogram ----
+    for (int i = tid; i < kTopkBins; i += blockDim.x) S.hist[i] = 0;
+    if (tid == 0) s_cc = 0;
+    __syncthreads();
+    for (int base = 0; base < n; base += 4 * kTopkThreads) {
+      const int i0 = base + 4 * tid;
+      float x[4];
+      if (vec && i0 + 3 < n) {
+        const float4 f = *reinterpret_cast<const float4*>(src + i0);
+        x[0] = f.x; x[1] = f.y; x[2] = f.z; x[3] = f.w;
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) x[q] = i0 + q < n ? src[i0 + q] : 0.f;
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const bool ok = i0 + q < n;
+        const unsigned act = __ballot_sync(0xffffffffu, ok);
+        if (ok) {
+          const uint32_t bin = float_key(x[q]) >> 20;
+          const unsigned peers = __match_any_sync(act, bin);   // lanes sharing this bin
+          if (lane == __ffs(peers) - 1) atomicAdd(&S.hist[bin], static_cast<uint32_t>(__popc(peers)));
+        }
+      }
+    }
+    __syncthreads();
+    int above;
+    const uint32_t b1 = static_cast<uint32_t>(topk_find_bin(S, kTopkBins, topk, &above));
+    const int in_b1 = static_cast<int>(S.hist[b1]);
+    __syncthreads();   // every thread has read the histogram before it is rewritten
+    if (above + in_b1 > cap) {
+      topk_row(src, n, topk, nullptr, out, S);
+      if (tid == 0) cnt[r] = topk;
+      continue;
+    }
+    // ---- pass 2: candidates at or above bin b1 ----
+    for (int base = 0; base < n; base += 4 * kTopkThreads) {
+      const int i0 = base + 4 * tid;
+      float x[4];
+      if (vec && i0 + 3 < n) {
+        const float4 f = *reinterpret_cast<const float4*>(src + i0);
+        x[0] = f.x; x[1] = f.y; x[2] = f.z; x[3] = f.w;
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) x[q] = i0 + q < n ? src[i0 + q] : 0.f;
+      }
+      uint32_t take = 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (i0 + q < n && (float_key(x[q]) >> 20) >= b1) take |= 1u << q;
+      int tot;
+      const int ex = warp_count_scan(__popc(take), &tot);
+      int slot = 0;
+      if (tot) {
+        if (lane == 0) slot = atomicAdd(&s_cc, tot);
+        slot = __shfl_sync(0xffffffffu, slot, 0) + ex;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (take & (1u << q)) {
+            c[slot] = (static_cast<uint64_t>(float_key(x[q])) << 32) | static_cast<uint32_t>(i0 + q);
+            ++slot;
+          }
+        }
+      }
+    }
+    __syncthreads();
+    topk_select_candidates(S, c, s_cc, b1, topk - above, sel, eqb, (n + 31) / 32, topk, out);
+    if (tid == 0) cnt[r] = topk;
+  }
 }
 
 // ---------------------------------------------------------------------------------------

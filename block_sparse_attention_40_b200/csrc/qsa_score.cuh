@@ -7,11 +7,13 @@
 // heads = 256 (prefill) or 1 token x 16 heads (decode) (B operand, loaded once per CTA),
 // K = 64.  The fp32 accumulator lives in TMEM (two buffers, so the epilogue of tile i
 // overlaps the MMA of tile i+1).  Epilogue: each thread owns one block row, reads its
-// 16 heads per token from TMEM, applies ReLU, weights by w and sums in fp32, and writes
-// the score if the block is a candidate of that token (b < floor(pos/4)).
+// 16 heads per token from TMEM, applies ReLU, weights by w and sums in fp32 (even and odd
+// heads as two partial sums), and writes the score if the block is a candidate of that token
+// (b < floor(pos/4)).
 //
 // Warp roles: warp 0 issues TMA, warp 1 allocates TMEM and issues MMAs (one thread),
 // the remaining warps run the epilogue.
+
 #pragma once
 
 #include "qsa_common.cuh"
@@ -73,6 +75,31 @@ struct ScoreWork {
   int32_t pos0;      // position (within the sequence) of token 0
   int64_t out_row0;  // score row of token 0
 };
+
+// s = sum_h w[h] * ReLU(d[h]) over the 16 heads of one (token, block): the even and the odd
+// heads accumulate as the two halves of packed f32x2 FMAs (each an fp32 fused multiply-add),
+// and the two partial sums are added at the end.  w: 16 weights in shared memory, 16-byte
+// aligned; d: the 16 fp32 accumulator words read from TMEM.
+__device__ __forceinline__ float head_weighted_relu_sum(const uint32_t* d, const float* w) {
+  const float4* w4 = reinterpret_cast<const float4*>(w);
+  uint64_t acc = 0ull;   // (+0.f, +0.f)
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float4 wq = w4[q];
+    uint64_t wa, wb, ra, rb;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(wa) : "f"(wq.x), "f"(wq.y));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(wb) : "f"(wq.z), "f"(wq.w));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(ra)
+        : "f"(fmaxf(__uint_as_float(d[4 * q]), 0.f)), "f"(fmaxf(__uint_as_float(d[4 * q + 1]), 0.f)));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(rb)
+        : "f"(fmaxf(__uint_as_float(d[4 * q + 2]), 0.f)), "f"(fmaxf(__uint_as_float(d[4 * q + 3]), 0.f)));
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(wa), "l"(ra));
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(wb), "l"(rb));
+  }
+  float even, odd;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(even), "=f"(odd) : "l"(acc));
+  return even + odd;
+}
 
 template <int NTOK>
 __device__ __forceinline__ ScoreWork<NTOK> score_work(const ScoreArgs& a) {
@@ -158,6 +185,7 @@ __global__ void __launch_bounds__(ScoreCfg<NTOK>::kThreads, 1)
   if constexpr (NTOK == 1) {
     for (int i = threadIdx.x; i < 4096; i += blockDim.x) sHist[i] = 0;
   }
+
   // weights of the tile's tokens, widened to fp32
   for (int i = threadIdx.x; i < NTOK * kIdxHeads; i += blockDim.x) {
     const int tok = i / kIdxHeads;
@@ -253,12 +281,7 @@ __global__ void __launch_bounds__(ScoreCfg<NTOK>::kThreads, 1)
 #pragma unroll
       for (int j = 0; j < kTokPerWarp; ++j) {
         const int tok = tok_base + j;
-        float s = 0.f;
-#pragma unroll
-        for (int h = 0; h < kIdxHeads; ++h) {
-          const float x = __uint_as_float(acc[j * kIdxHeads + h]);
-          s = fmaf(sW[tok * kIdxHeads + h], fmaxf(x, 0.f), s);
-        }
+        const float s = head_weighted_relu_sum(acc + j * kIdxHeads, sW + tok * kIdxHeads);
         const int pos = wk.pos0 + tok;
         const bool valid = tok < wk.ntok && blk < pos / kBlock;
         if (valid) args.scores[(wk.out_row0 + tok) * args.ld + blk] = s;

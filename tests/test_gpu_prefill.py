@@ -86,3 +86,55 @@ def test_64k_sampled():
     idx, cnt, out = _run(p)
     rows = rows_sample(65536, 4096, seed=3)
     prefill_oracle_check(p, idx, cnt, out, rows)
+
+
+def _select_check(p, rows, exact=False, chunk=0):
+    d = p.to(DEV)
+    ctx = qsa.Prefill(p.cu_seqlens, DEV, p.topk, 0, chunk)
+    idx, cnt = ctx.select(d.q_idx, d.k_idx, d.w)
+    torch.cuda.synchronize()
+    assert ctx.device_error() == ("QSA_OK", 0)
+    return prefill_oracle_check(p, idx, cnt, None, rows, exact_sel=exact)
+
+
+@pytest.mark.parametrize("topk", [513, 640])
+def test_selection_large_budgets_drift(topk):
+    # budgets above 512 blocks on keys that drift along the sequence, so scores trend with
+    # the block index
+    p = W.custom_prefill([9000, 2222], topk=topk, kind="drift", seed=topk)
+    T = int(p.cu_seqlens[-1])
+    _select_check(p, rows_sample(T, 1536, seed=4, cu=p.cu_seqlens.tolist()))
+
+
+def test_selection_budget_700_small_chunks():
+    # a budget of 700 blocks with score chunks of 2048 rows
+    p = W.custom_prefill([5000, 3001], topk=700, kind="normal", seed=7)
+    T = int(p.cu_seqlens[-1])
+    _select_check(p, rows_sample(T, 1536, seed=3, cu=p.cu_seqlens.tolist()), chunk=2048)
+
+
+def test_selection_all_scores_equal():
+    # w = 0 makes every score 0: each row selects its lowest topk block indices
+    p = W.custom_prefill([7000, 50, 3], topk=512, kind="normal", seed=9)
+    p.w.zero_()
+    T = int(p.cu_seqlens[-1])
+    _select_check(p, rows_sample(T, 1024, seed=5, cu=p.cu_seqlens.tolist()), exact=True)
+
+
+def test_selection_integer_scores_many_ties_small_budget():
+    # small-integer indexer inputs with a budget of 5 blocks: long runs of equal scores at
+    # the threshold, resolved toward lower block indices
+    p = W.custom_prefill([4100, 999], topk=5, kind="int", seed=10)
+    T = int(p.cu_seqlens[-1])
+    _select_check(p, rows_sample(T, 1024, seed=6, cu=p.cu_seqlens.tolist()), exact=True)
+
+
+@pytest.mark.slow
+def test_selection_rows_beyond_65536_blocks():
+    # rows of more than 65,536 candidate blocks (positions past 262,144 tokens)
+    L = 266_300
+    p = W.custom_prefill([L], topk=512, kind="normal", seed=11, device=DEV)
+    rows = np.concatenate([rows_sample(L, 256, seed=7), np.arange(L - 64, L - 8),
+                           np.arange(262_140, 262_160)])
+    rows = np.unique(rows)
+    _select_check(p, rows)
