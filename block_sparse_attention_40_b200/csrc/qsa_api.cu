@@ -691,11 +691,23 @@ qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, 
     if (!make_tmap(&tm_qidx, q_idx, 2, dq, sk, bq)) return QSA_ERR_CUDA;
     using C = ScoreCfg<1>;
     if (!set_smem(k_index_score<1>, C::kSmemBytes)) return QSA_ERR_CUDA;
+    // split each sequence's M-tiles over CTAs: fewest waves x tiles per CTA over the SMs'
+    // CTA slots, counting a fixed cost of two tiles per CTA for its setup and histogram flush
     const int total_mt = std::max(1, (max_nc_now + 127) / 128);
-    int splits = std::max(1, (2 * sms + g.B - 1) / g.B);
-    splits = std::min(splits, total_mt);
-    const int per = (total_mt + splits - 1) / splits;
-    splits = (total_mt + per - 1) / per;
+    const int64_t slots = int64_t(sms) * C::kCtasPerSm;
+    int splits = 1, per = total_mt;
+    int64_t best = -1;
+    for (int sp = 1; sp <= std::min(total_mt, 256); ++sp) {
+      const int pr = (total_mt + sp - 1) / sp;
+      const int se = (total_mt + pr - 1) / pr;
+      const int64_t waves = (int64_t(g.B) * se + slots - 1) / slots;
+      const int64_t cost = waves * (pr + 2);
+      if (best < 0 || cost < best) {
+        best = cost;
+        splits = se;
+        per = pr;
+      }
+    }
     ScoreArgs a{};
     a.len = cache->len;
     a.splits = splits;

@@ -27,7 +27,8 @@ struct ScoreCfg {
   static constexpr int kAccCols = kN < 32 ? 32 : kN;      // TMEM columns per accumulator
   static constexpr int kNumAcc = NTOK == 16 ? 2 : 4;
   static constexpr int kTmemCols = kAccCols * kNumAcc;    // 512 / 128
-  static constexpr int kStages = NTOK == 16 ? 4 : 8;
+  static constexpr int kStages = NTOK == 16 ? 4 : 5;     // decode: 2 CTAs per SM
+  static constexpr int kCtasPerSm = NTOK == 16 ? 1 : 2;
   static constexpr int kEpiWarps = NTOK == 16 ? 8 : 4;
   static constexpr int kThreads = 64 + 32 * kEpiWarps;
   static constexpr int kABytes = 128 * kIdxDim * 2;       // 16 KB
@@ -41,6 +42,8 @@ struct ScoreCfg {
   static constexpr int kHistBytes = NTOK == 1 ? 4096 * 4 : 0;
   static constexpr int kSmemBytes = kHistOff + kHistBytes + 1024;  // + align slack
   static constexpr uint32_t kIdesc = idesc_bf16_f32(128, kN, 0, 0);
+  static_assert(kCtasPerSm * (kSmemBytes + 1024) <= 228 * 1024, "shared memory per SM");
+  static_assert(kCtasPerSm * kTmemCols <= 512, "TMEM columns per SM");
 };
 
 struct ScoreArgs {
@@ -141,7 +144,7 @@ __device__ __forceinline__ ScoreWork<NTOK> score_work(const ScoreArgs& a) {
 }
 
 template <int NTOK>
-__global__ void __launch_bounds__(ScoreCfg<NTOK>::kThreads, 1)
+__global__ void __launch_bounds__(ScoreCfg<NTOK>::kThreads, ScoreCfg<NTOK>::kCtasPerSm)
     k_index_score(const __grid_constant__ CUtensorMap tmap_kbar,
                   const __grid_constant__ CUtensorMap tmap_qidx, ScoreArgs args) {
   using C = ScoreCfg<NTOK>;
