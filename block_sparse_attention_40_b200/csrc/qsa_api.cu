@@ -346,7 +346,10 @@ qsa_status decode_geom(const qsa_cache* c, const qsa_params& p, DecodeGeom* g) {
   g->topk = p.topk_blocks;
   g->max_nc = (c->capacity - 1) / 4;
   g->ld = std::max<int64_t>(4, round_up(std::max(g->max_nc, 1), 4));
-  g->splits = p.decode_splits > 0 ? p.decode_splits : 4;
+  // default: as many splits as keep one wave of (sequence, KV head, split) CTAs on the SMs;
+  // a CTA's fixed costs (setup, pipeline fill, partial write) favour fewer, longer CTAs
+  g->splits = p.decode_splits > 0 ? p.decode_splits
+                                  : std::max(1, std::min(64, num_sms() / (2 * g->B)));
   if (g->splits > 64) return QSA_ERR_INVALID_ARG;
   g->pl = make_plan_layout(1, g->topk);
   Carver cv;

@@ -81,8 +81,8 @@ typedef struct {
   int32_t topk_blocks;     /* budget k in blocks, 1..QSA_MAX_TOPK (512 on the pages) */
   int32_t rows_per_tile;   /* prefill attention: query tokens packed into one 128-row
                               tensor-core tile (1..10); 0 = library default */
-  int32_t decode_splits;   /* decode attention: key splits per (sequence, KV head);
-                              0 = library default */
+  int32_t decode_splits;   /* decode attention: key splits per (sequence, KV head), 1..64;
+                              0 = library default (one wave of CTAs: SMs / (2 x batch)) */
   int32_t score_chunk_rows;/* prefill: query rows scored per pass (bounds the score
                               buffer in the workspace); 0 = library default */
 } qsa_params;
