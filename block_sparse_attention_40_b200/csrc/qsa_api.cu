@@ -275,11 +275,10 @@ qsa_status run_attention(const void* q, const void* k, const void* v, const int3
   {
     const int mwords = g.pl.umax / 32;
     const int smem = (2 * g.max_words + g.R * mwords) * 4;
-    if (!set_smem(k_attn_plan<false>, smem)) return QSA_ERR_CUDA;
+    if (!set_smem(k_attn_plan, smem)) return QSA_ERR_CUDA;
     const int grid = std::min(g.attn_tiles, num_sms() * 8);
-    k_attn_plan<false><<<grid, kPlanThreads, smem, s>>>(idx, cnt, g.topk, meta, num_seqs, nullptr,
-                                                        g.attn_tiles, g.pl, g.max_words, plan,
-                                                        dev_status(ws));
+    k_attn_plan<<<grid, kPlanThreads, smem, s>>>(idx, cnt, g.topk, meta, num_seqs, g.attn_tiles,
+                                                 g.pl, g.max_words, plan, dev_status(ws));
     QSA_CHECK_LAUNCH();
   }
   AttnMaps maps;
@@ -627,16 +626,10 @@ qsa_status qsa_append_kv(const qsa_cache* cache, const void* k, const void* v, c
   p.st = DevStatus{nullptr};
   const int sms = num_sms();
   {
-    const int64_t n = static_cast<int64_t>(p.batch) * n_new * 32;
+    const int slots = (n_new + 3) / 4 + 1;   // blocks a sequence's new tokens can touch
+    const int64_t n = static_cast<int64_t>(p.batch) * n_new * 32 + static_cast<int64_t>(p.batch) * slots * 8;
     const int grid = static_cast<int>(std::min<int64_t>((n + 255) / 256, int64_t(sms) * 16));
-    k_append_kv_copy<<<grid, 256, 0, s>>>(p);
-    QSA_CHECK_LAUNCH();
-  }
-  {
-    const int slots = (n_new + 3) / 4 + 1;
-    const int64_t n = static_cast<int64_t>(p.batch) * slots * 8;
-    const int grid = static_cast<int>(std::min<int64_t>((n + 255) / 256, int64_t(sms) * 16));
-    k_append_kbar<<<grid, 256, 0, s>>>(p, slots);
+    k_append<<<grid, 256, 0, s>>>(p, slots);
     QSA_CHECK_LAUNCH();
   }
   k_append_len<<<(p.batch + 255) / 256, 256, 0, s>>>(cache->len, counts, n_new, p.batch);
@@ -734,19 +727,10 @@ qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, 
     QSA_CHECK_LAUNCH();
     const int smem = g.finish_smem();
     if (!set_smem(k_topk_finish, smem)) return QSA_ERR_CUDA;
+    // also writes each sequence's attention plan record
     k_topk_finish<<<g.B, kTopkThreads, smem, s>>>(scores, g.ld, n_c, g.topk, g.cand_cap,
                                                    std::max(g.max_nc, 1), hist, cand_cnt, cand,
-                                                   idx, cnt);
-    QSA_CHECK_LAUNCH();
-  }
-  // union plan (one token per tile)
-  {
-    const int max_words = (g.cap - 1) / 4 / 32 + 1;
-    const int mwords = g.pl.umax / 32;
-    const int smem = (2 * max_words + mwords) * 4;
-    if (!set_smem(k_attn_plan<true>, smem)) return QSA_ERR_CUDA;
-    k_attn_plan<true><<<std::min(g.B, sms * 8), kPlanThreads, smem, s>>>(
-        idx, cnt, g.topk, nullptr, 0, cache->len, g.B, g.pl, max_words, plan, dev_status(ws));
+                                                   idx, cnt, cache->len, g.pl, plan);
     QSA_CHECK_LAUNCH();
   }
   // a6: split attention + combine
@@ -777,13 +761,16 @@ qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, 
     a.part_l = reinterpret_cast<float*>(ws + g.o_pl);
     a.st = dev_status(ws);
     dim3 grid(g.B, 2, g.splits);
+    a.out = reinterpret_cast<__nv_bfloat16*>(out);   // written directly with one split
     k_sparse_attn<<<grid, AttnCfg::kThreads, AttnCfg::kSmemBytes, s>>>(maps, a);
     QSA_CHECK_LAUNCH();
-    const int warps = g.B * kHeads;
-    k_decode_combine<<<(warps * 32 + 255) / 256, 256, 0, s>>>(a.part_o, a.part_m, a.part_l, g.B,
-                                                              g.splits,
-                                                              reinterpret_cast<__nv_bfloat16*>(out));
-    QSA_CHECK_LAUNCH();
+    if (g.splits > 1) {
+      const int warps = g.B * kHeads;
+      k_decode_combine<<<(warps * 32 + 255) / 256, 256, 0, s>>>(a.part_o, a.part_m, a.part_l,
+                                                                g.B, g.splits,
+                                                                reinterpret_cast<__nv_bfloat16*>(out));
+      QSA_CHECK_LAUNCH();
+    }
   }
   return QSA_OK;
 }

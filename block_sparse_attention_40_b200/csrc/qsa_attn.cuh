@@ -69,7 +69,7 @@ struct AttnArgs {
   int32_t decode;          // 1: decode (tile = sequence, KV from the block cache)
   int32_t splits;          // chunk splits per tile (decode), 1 for prefill
   int64_t cap_blocks;      // decode: capacity / 4
-  __nv_bfloat16* out;      // prefill: [T][24][128]
+  __nv_bfloat16* out;      // prefill: [T][24][128]; decode with one split: [B][24][128]
   float* part_o;           // decode: [B][2][splits][12][128]
   float* part_m;           // decode: [B][2][splits][12]
   float* part_l;
@@ -483,7 +483,7 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
           tmem_ld32(to + 32, ov + 32);
           tmem_wait_ld();
           if (row_ok) {
-            if (!args.decode) {
+            if (!args.decode || args.splits == 1) {   // one split: the final output directly
               const float inv = l_all > 0.f ? 1.f / l_all : 0.f;
               __nv_bfloat16* o = args.out + ((tok_row0 + tr) * kHeads + g * kGroup + hr) * kHeadDim +
                                  64 * wg;

@@ -212,23 +212,21 @@ __device__ __forceinline__ int append_count(const AppendParams& p, int b) {
   return c < 0 ? 0 : (c > p.n_new ? p.n_new : c);
 }
 
-// Copies: one thread per 16 bytes of K or V.
-__global__ void k_append_kv_copy(AppendParams p) {
+// Copies: one work item per 16 bytes of K and V (items 0 .. batch * n_new * 32).
+__device__ __forceinline__ void append_copy_item(const AppendParams& p, int64_t i) {
   const int64_t per_tok = 2 * 16;                       // 2 heads x 16 units of 16 B
-  const int64_t n = static_cast<int64_t>(p.batch) * p.n_new * per_tok;
   const int64_t cap_blk = p.capacity / kBlock;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x) {
+  {
     const int b = static_cast<int>(i / (static_cast<int64_t>(p.n_new) * per_tok));
     const int64_t rem = i - static_cast<int64_t>(b) * p.n_new * per_tok;
     const int j = static_cast<int>(rem / per_tok);
     const int g = static_cast<int>((rem / 16) & 1);
     const int u = static_cast<int>(rem & 15);
-    if (j >= append_count(p, b)) continue;
+    if (j >= append_count(p, b)) return;
     const int64_t pos = static_cast<int64_t>(p.len[b]) + j;
     if (pos >= p.capacity) {
       report_error(p.st, kErrDevice, 200);
-      continue;
+      return;
     }
     const int64_t dst = ((((static_cast<int64_t>(b) * 2 + g) * cap_blk + pos / 4) * 4 + pos % 4) *
                          16) + u;
@@ -248,24 +246,24 @@ __global__ void k_append_kv_copy(AppendParams p) {
   }
 }
 
-// Compressed keys: one thread per (sequence, touched block, 8-dim slice).  Slot 0 of each
-// sequence handles the first and the last touched block; slots 1.. the complete middle ones.
-__global__ void k_append_kbar(AppendParams p, int max_blocks_touched) {
+// Compressed keys: one work item per (sequence, touched block, 8-dim slice), items 0 ..
+// batch * max_blocks_touched * 8.  Slot 0 of each sequence handles the first and the last
+// touched block; slots 1.. the complete middle ones.
+__device__ __forceinline__ void append_kbar_item(const AppendParams& p, int64_t i,
+                                                 int max_blocks_touched) {
   const int64_t slots = static_cast<int64_t>(max_blocks_touched);
-  const int64_t n = static_cast<int64_t>(p.batch) * slots * 8;
   const int64_t cap_blk = p.capacity / kBlock;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x) {
+  {
     const int b = static_cast<int>(i / (slots * 8));
     const int64_t slot = (i / 8) % slots;
     const int part = static_cast<int>(i & 7);
     const int cnt = append_count(p, b);
-    if (cnt == 0) continue;
+    if (cnt == 0) return;
     const int64_t L0 = p.len[b];
     const int64_t L1 = L0 + cnt;
     if (L1 > p.capacity) {
       if (slot == 0 && part == 0) report_error(p.st, kErrDevice, 201);
-      continue;
+      return;
     }
     const int64_t jf = L0 / 4, jl = (L1 - 1) / 4;
     const uint4* kin = p.k_idx + static_cast<int64_t>(b) * p.n_new * 8 + part;  // token j at +8j
@@ -320,10 +318,22 @@ __global__ void k_append_kbar(AppendParams p, int max_blocks_touched) {
       }
     } else {
       const int64_t j = jf + slot;       // middle blocks jf+1 .. jl-1 are complete and new
-      if (j >= jl) continue;
+      if (j >= jl) return;
       add_tokens(acc, 4 * j, 4 * j + 4, true);
       finish(acc, j, true);
     }
+  }
+}
+
+// K/V copies and compressed-key updates in one launch (both read the lengths before the
+// append); k_append_len then advances the lengths.
+__global__ void k_append(AppendParams p, int max_blocks_touched) {
+  const int64_t n_copy = static_cast<int64_t>(p.batch) * p.n_new * 32;
+  const int64_t n_kbar = static_cast<int64_t>(p.batch) * max_blocks_touched * 8;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n_copy + n_kbar;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    if (i < n_copy) append_copy_item(p, i);
+    else append_kbar_item(p, i - n_copy, max_blocks_touched);
   }
 }
 
@@ -332,6 +342,56 @@ __global__ void k_append_len(int32_t* len, const int32_t* counts, int32_t n_new,
     int c = counts ? counts[b] : n_new;
     c = c < 0 ? 0 : (c > n_new ? n_new : c);
     len[b] += c;
+  }
+}
+
+// Attention plan.  A tile is up to R consecutive query tokens of one sequence (R = 1 for
+// decode, whose records the decode top-k writes directly).  The tile's key set is the union U
+// of its tokens' selected blocks and their own blocks, in ascending block order.  For every token r and every 32-block chunk q of the
+// union, mask[r][q] has bit u set when union block 32q+u is selected by r or is r's own
+// block; tail[r] is the union position of r's own block.
+struct PlanLayout {
+  int32_t R;         // tokens per tile
+  int32_t umax;      // union capacity per tile (multiple of 32)
+  int64_t stride;    // int32 entries per tile record
+  // record: [0] = U, [1] = number of tokens, [2] = position of token 0 in its sequence,
+  //         [3] unused, [4..4+R) = union position of each token's own block,
+  //         [4+R .. 4+R+umax) = union block ids, then R * (umax/32) mask words
+  __host__ __device__ int64_t tail_off() const { return 4; }
+  __host__ __device__ int64_t union_off() const { return 4 + R; }
+  __host__ __device__ int64_t mask_off() const { return 4 + R + umax; }
+};
+
+__host__ __device__ inline PlanLayout make_plan_layout(int R, int topk) {
+  PlanLayout pl;
+  pl.R = R;
+  pl.umax = ((R * (topk + 1)) + 31) / 32 * 32;
+  pl.stride = 4 + R + pl.umax + static_cast<int64_t>(R) * (pl.umax / 32);
+  pl.stride = (pl.stride + 3) / 4 * 4;   // 16-byte aligned records
+  return pl;
+}
+
+// Decode: the plan record of a one-token tile, written straight from the token's selection
+// sel[0 .. k) (ascending, all below its own block c): the union is the selection followed by
+// c, every union block is attended, and c sits at union position k.  Called by all threads of
+// a CTA after sel is complete.
+__device__ __forceinline__ void write_decode_plan(int32_t* rec, const PlanLayout& pl,
+                                                  const int32_t* sel, int k, int c, int p) {
+  const int U = k + 1;
+  int32_t* uni = rec + pl.union_off();
+  for (int j = threadIdx.x; j < k; j += blockDim.x) uni[j] = sel[j];
+  uint32_t* m = reinterpret_cast<uint32_t*>(rec + pl.mask_off());
+  const int nq = (U + 31) / 32;
+  for (int q = threadIdx.x; q < nq; q += blockDim.x) {
+    const int rem = U - 32 * q;
+    m[q] = rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u);
+  }
+  if (threadIdx.x == 0) {
+    uni[k] = c;
+    rec[0] = U;
+    rec[1] = 1;
+    rec[2] = p;
+    rec[pl.tail_off()] = k;
   }
 }
 
@@ -675,10 +735,12 @@ __device__ __forceinline__ void topk_select_candidates(TopkShared& S, const uint
 }
 
 // Shared memory: TopkShared, then cap candidates (uint64), then two bitmaps of n_max bits.
+// Besides idx/cnt, the finish kernel writes each row's attention plan record (one-token tile).
 __global__ void __launch_bounds__(kTopkThreads) k_topk_finish(
     const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_c, int topk,
     int cap, int n_max, const uint32_t* __restrict__ hist, const int32_t* __restrict__ cand_cnt,
-    const uint64_t* __restrict__ cand, int32_t* __restrict__ idx, int32_t* __restrict__ cnt) {
+    const uint64_t* __restrict__ cand, int32_t* __restrict__ idx, int32_t* __restrict__ cnt,
+    const int32_t* __restrict__ len, PlanLayout pl, int32_t* __restrict__ plan) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   TopkShared& S = *reinterpret_cast<TopkShared*>(smem_raw);
   uint64_t* c = reinterpret_cast<uint64_t*>(smem_raw + kTopkSharedBytes);
@@ -689,9 +751,13 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk_finish(
   const int r = blockIdx.x;
   const int n = n_c[r];
   int32_t* out = idx + static_cast<int64_t>(r) * topk;
+  int32_t* rec = plan + static_cast<int64_t>(r) * pl.stride;
+  const int p = len[r] - 1;
   if (n <= topk) {
     for (int i = tid; i < topk; i += blockDim.x) out[i] = i < n ? i : -1;
     if (tid == 0) cnt[r] = n < 0 ? 0 : n;
+    __syncthreads();
+    write_decode_plan(rec, pl, out, n < 0 ? 0 : n, n < 0 ? 0 : n, p);
     return;
   }
   const uint32_t* h = hist + static_cast<int64_t>(r) * 4096;
@@ -706,11 +772,15 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk_finish(
     // the candidates did not fit: full-row radix select on the scores in global memory
     topk_row(scores + static_cast<int64_t>(r) * ld, n, topk, h, out, S);
     if (tid == 0) cnt[r] = topk;
+    __syncthreads();
+    write_decode_plan(rec, pl, out, topk, n, p);
     return;
   }
   for (int i = tid; i < C; i += blockDim.x) c[i] = cand[static_cast<int64_t>(r) * cap + i];
   topk_select_candidates(S, c, C, b1, topk - above, sel, eqb, (n + 31) / 32, topk, out);
   if (tid == 0) cnt[r] = topk;
+  __syncthreads();
+  write_decode_plan(rec, pl, out, topk, n, p);
 }
 
 // Step a3 on score rows, one CTA per row (grid-strided): pass 1 reads the row and builds the
@@ -814,40 +884,13 @@ __global__ void __launch_bounds__(kTopkThreads, 4) k_topk(const float* __restric
 }
 
 // ---------------------------------------------------------------------------------------
-// Attention plan.  A tile is up to R consecutive query tokens of one sequence (R = 1 for
-// decode).  The tile's key set is the union U of its tokens' selected blocks and their own
-// blocks, in ascending block order.  For every token r and every 32-block chunk q of the
-// union, mask[r][q] has bit u set when union block 32q+u is selected by r or is r's own
-// block; tail[r] is the union position of r's own block.
-struct PlanLayout {
-  int32_t R;         // tokens per tile
-  int32_t umax;      // union capacity per tile (multiple of 32)
-  int64_t stride;    // int32 entries per tile record
-  // record: [0] = U, [1] = number of tokens, [2] = position of token 0 in its sequence,
-  //         [3] unused, [4..4+R) = union position of each token's own block,
-  //         [4+R .. 4+R+umax) = union block ids, then R * (umax/32) mask words
-  __host__ __device__ int64_t tail_off() const { return 4; }
-  __host__ __device__ int64_t union_off() const { return 4 + R; }
-  __host__ __device__ int64_t mask_off() const { return 4 + R + umax; }
-};
-
-__host__ __device__ inline PlanLayout make_plan_layout(int R, int topk) {
-  PlanLayout pl;
-  pl.R = R;
-  pl.umax = ((R * (topk + 1)) + 31) / 32 * 32;
-  pl.stride = 4 + R + pl.umax + static_cast<int64_t>(R) * (pl.umax / 32);
-  pl.stride = (pl.stride + 3) / 4 * 4;   // 16-byte aligned records
-  return pl;
-}
-
 constexpr int kPlanThreads = 256;
 
 // kDecode: tile = sequence b, single token at p = len[b]-1, selection rows idx[b].
-template <bool kDecode>
 __global__ void __launch_bounds__(kPlanThreads) k_attn_plan(
     const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt, int topk,
-    const SeqMeta* __restrict__ meta, int num_seqs, const int32_t* __restrict__ len,
-    int num_tiles, PlanLayout pl, int max_words, int32_t* __restrict__ plan, DevStatus st) {
+    const SeqMeta* __restrict__ meta, int num_seqs, int num_tiles, PlanLayout pl, int max_words,
+    int32_t* __restrict__ plan, DevStatus st) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   uint32_t* bitmap = reinterpret_cast<uint32_t*>(smem_raw);          // max_words
   int* wpref = reinterpret_cast<int*>(bitmap + max_words);            // max_words
@@ -859,19 +902,13 @@ __global__ void __launch_bounds__(kPlanThreads) k_attn_plan(
   const int mwords = pl.umax / 32;
   for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
     if (tid == 0) {
-      if (kDecode) {
-        s_row0 = tile;
-        s_pos0 = len[tile] - 1;
-        s_ntok = 1;
-      } else {
-        const int s = find_seq_of_tile<true>(meta, num_seqs, tile);
-        const int lt = tile - meta[s].attn_tile0;
-        const int p0 = lt * pl.R;
-        s_pos0 = p0;
-        s_row0 = meta[s].tok0 + p0;
-        const int rem = meta[s].len - p0;
-        s_ntok = rem < pl.R ? rem : pl.R;
-      }
+      const int s = find_seq_of_tile<true>(meta, num_seqs, tile);
+      const int lt = tile - meta[s].attn_tile0;
+      const int p0 = lt * pl.R;
+      s_pos0 = p0;
+      s_row0 = meta[s].tok0 + p0;
+      const int rem = meta[s].len - p0;
+      s_ntok = rem < pl.R ? rem : pl.R;
     }
     __syncthreads();
     const int ntok = s_ntok, pos0 = s_pos0;
