@@ -162,6 +162,35 @@ std::atomic<uint64_t> g_launches{0};
     }                                                       \
   } while (0)
 
+// Launches a kernel with programmatic stream serialization: it may start while the kernel
+// before it in the stream finishes; the kernel waits (pdl_wait) before it uses its inputs.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+#define QSA_CHECK_PDL(expr)                                  \
+  do {                                                       \
+    g_launches.fetch_add(1, std::memory_order_relaxed);      \
+    cudaError_t e_ = (expr);                                 \
+    if (e_ != cudaSuccess) {                                 \
+      fprintf(stderr, "qsa: launch failed: %s (%s:%d)\n",   \
+              cudaGetErrorString(e_), __FILE__, __LINE__);   \
+      return QSA_ERR_CUDA;                                   \
+    }                                                        \
+  } while (0)
+
 template <typename K>
 bool set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
@@ -673,8 +702,13 @@ qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, 
   uint64_t* cand = reinterpret_cast<uint64_t*>(ws + g.o_cand);
   const int sms = num_sms();
   const int max_nc_now = (max_len - 1) / 4;
-  if (cudaMemsetAsync(hist, 0, static_cast<size_t>(g.B) * (kTopkBins + 1) * 4, s) != cudaSuccess)
-    return QSA_ERR_CUDA;
+  // the decode kernels form one chain of programmatic dependent launches (each waits for the
+  // one before it); the first also follows the caller's last kernel (the append) that way
+  {
+    const int64_t words = static_cast<int64_t>(g.B) * (kTopkBins + 1);
+    const int grid = static_cast<int>(std::min<int64_t>((words + 255) / 256, int64_t(sms) * 4));
+    QSA_CHECK_PDL(launch_pdl(k_zero_words, dim3(grid), dim3(256), 0, s, hist, words));
+  }
   // a2: scores, with the first radix digit's histogram of every row (one token x 16 heads per sequence, split over M-tiles)
   {
     CUtensorMap tm_kbar, tm_qidx;
@@ -715,23 +749,27 @@ qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, 
     a.scores = scores;
     a.ld = g.ld;
     a.st = dev_status(ws);
-    k_index_score<1><<<g.B * splits, C::kThreads, C::kSmemBytes, s>>>(tm_kbar, tm_qidx, a);
-    QSA_CHECK_LAUNCH();
+    QSA_CHECK_PDL(launch_pdl(k_index_score<1>, dim3(g.B * splits), dim3(C::kThreads),
+                             C::kSmemBytes, s, tm_kbar, tm_qidx, a));
   }
   // a3: top-k: candidates at or above the threshold bin, then the exact select per row
   {
     // one pass of 4096 scores per CTA
     const int parts = std::max(1, (max_nc_now + 4095) / 4096);
-    k_topk_collect<<<g.B * parts, kCandThreads, 0, s>>>(scores, g.ld, n_c, g.topk, parts,
-                                                         g.cand_cap, hist, cand_cnt, cand);
-    QSA_CHECK_LAUNCH();
+    QSA_CHECK_PDL(launch_pdl(k_topk_collect, dim3(g.B * parts), dim3(kCandThreads), 0, s,
+                             static_cast<const float*>(scores), g.ld,
+                             static_cast<const int32_t*>(n_c), g.topk, parts, g.cand_cap,
+                             static_cast<const uint32_t*>(hist), cand_cnt, cand));
     const int smem = g.finish_smem();
     if (!set_smem(k_topk_finish, smem)) return QSA_ERR_CUDA;
     // also writes each sequence's attention plan record
-    k_topk_finish<<<g.B, kTopkThreads, smem, s>>>(scores, g.ld, n_c, g.topk, g.cand_cap,
-                                                   std::max(g.max_nc, 1), hist, cand_cnt, cand,
-                                                   idx, cnt, cache->len, g.pl, plan);
-    QSA_CHECK_LAUNCH();
+    QSA_CHECK_PDL(launch_pdl(k_topk_finish, dim3(g.B), dim3(kTopkThreads), smem, s,
+                             static_cast<const float*>(scores), g.ld,
+                             static_cast<const int32_t*>(n_c), g.topk, g.cand_cap,
+                             std::max(g.max_nc, 1), static_cast<const uint32_t*>(hist),
+                             static_cast<const int32_t*>(cand_cnt),
+                             static_cast<const uint64_t*>(cand), idx, cnt,
+                             static_cast<const int32_t*>(cache->len), g.pl, plan));
   }
   // a6: split attention + combine
   {
@@ -762,14 +800,15 @@ qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, 
     a.st = dev_status(ws);
     dim3 grid(g.B, 2, g.splits);
     a.out = reinterpret_cast<__nv_bfloat16*>(out);   // written directly with one split
-    k_sparse_attn<<<grid, AttnCfg::kThreads, AttnCfg::kSmemBytes, s>>>(maps, a);
-    QSA_CHECK_LAUNCH();
+    QSA_CHECK_PDL(launch_pdl(k_sparse_attn, grid, dim3(AttnCfg::kThreads), AttnCfg::kSmemBytes,
+                             s, maps, a));
     if (g.splits > 1) {
       const int warps = g.B * kHeads;
-      k_decode_combine<<<(warps * 32 + 255) / 256, 256, 0, s>>>(a.part_o, a.part_m, a.part_l,
-                                                                g.B, g.splits,
-                                                                reinterpret_cast<__nv_bfloat16*>(out));
-      QSA_CHECK_LAUNCH();
+      QSA_CHECK_PDL(launch_pdl(k_decode_combine, dim3((warps * 32 + 255) / 256), dim3(256), 0, s,
+                               static_cast<const float*>(a.part_o),
+                               static_cast<const float*>(a.part_m),
+                               static_cast<const float*>(a.part_l), g.B, g.splits,
+                               reinterpret_cast<__nv_bfloat16*>(out)));
     }
   }
   return QSA_OK;

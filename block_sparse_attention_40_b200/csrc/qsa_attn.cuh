@@ -181,6 +181,8 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
 
+  pdl_trigger();
+  pdl_wait();   // decode: the plan records come from the kernel before
   const int g = blockIdx.y;
   const int split = blockIdx.z;
   const int tile = blockIdx.x;

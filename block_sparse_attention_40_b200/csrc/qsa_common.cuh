@@ -147,6 +147,15 @@ __device__ __forceinline__ void named_barrier_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// ---- programmatic dependent launch -------------------------------------------------------
+// A kernel launched with programmatic stream serialization may start while the kernel before
+// it in the stream is still running.  pdl_wait blocks until that kernel has completed and its
+// memory is visible (and, since every kernel of such a chain waits, all earlier ones too); a
+// kernel reads or writes nothing the earlier kernels touch before it.  pdl_trigger lets the
+// next kernel start early.  Both are no-ops for a kernel launched normally.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;"); }
+
 // ---- TMA (no multicast anywhere in this library) ----------------------------------------
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(m) : "memory");

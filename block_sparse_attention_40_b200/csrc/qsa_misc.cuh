@@ -337,6 +337,15 @@ __global__ void k_append(AppendParams p, int max_blocks_touched) {
   }
 }
 
+// Zeroes n 32-bit words (the decode histograms and candidate counters).
+__global__ void k_zero_words(uint32_t* __restrict__ p, int64_t n) {
+  pdl_trigger();
+  pdl_wait();
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    p[i] = 0u;
+}
+
 __global__ void k_append_len(int32_t* len, const int32_t* counts, int32_t n_new, int batch) {
   for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < batch; b += gridDim.x * blockDim.x) {
     int c = counts ? counts[b] : n_new;
@@ -601,6 +610,8 @@ __global__ void __launch_bounds__(kCandThreads) k_topk_collect(
     const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_c, int topk,
     int parts, int cap, const uint32_t* __restrict__ hist, int32_t* __restrict__ cand_cnt,
     uint64_t* __restrict__ cand) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int sh[40];
   __shared__ int s_base;
   const int r = blockIdx.x / parts, part = blockIdx.x % parts;
@@ -741,6 +752,8 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk_finish(
     int cap, int n_max, const uint32_t* __restrict__ hist, const int32_t* __restrict__ cand_cnt,
     const uint64_t* __restrict__ cand, int32_t* __restrict__ idx, int32_t* __restrict__ cnt,
     const int32_t* __restrict__ len, PlanLayout pl, int32_t* __restrict__ plan) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   TopkShared& S = *reinterpret_cast<TopkShared*>(smem_raw);
   uint64_t* c = reinterpret_cast<uint64_t*>(smem_raw + kTopkSharedBytes);
@@ -1019,6 +1032,8 @@ __global__ void __launch_bounds__(kPlanThreads) k_attn_plan(
 __global__ void k_decode_combine(const float* __restrict__ part_o, const float* __restrict__ part_m,
                                  const float* __restrict__ part_l, int batch, int splits,
                                  __nv_bfloat16* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= batch * kHeads) return;

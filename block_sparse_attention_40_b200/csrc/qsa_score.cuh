@@ -164,6 +164,8 @@ __global__ void __launch_bounds__(ScoreCfg<NTOK>::kThreads, ScoreCfg<NTOK>::kCta
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
 
+  pdl_trigger();
+  pdl_wait();   // decode: the lengths, keys and weights come from earlier kernels
   const ScoreWork<NTOK> wk = score_work<NTOK>(args);
   if (wk.n_mtiles <= 0) return;   // uniform over the CTA
 
