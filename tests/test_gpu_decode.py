@@ -165,3 +165,26 @@ def test_decode_256k_four_sequences():
 def test_decode_1m_incremental():
     spec = W.decode_spec("decode1m")
     _decode_session(spec, check_seqs=[0, 3], steps=4, device_gen=True)
+
+
+def test_decode_batch_of_40_mixed_contexts():
+    # 40 sequences of 3,000..4,799 tokens: each sequence keeps its own selection and output
+    ctx = tuple(3000 + (373 * i) % 1800 for i in range(40))
+    spec = W.small_decode_spec(batch=40, context=ctx, capacity=4900, topk=128, steps=2, seed=24)
+    _decode_session(spec, check_seqs=[0, 17, 39], steps=2)
+
+
+def test_decode_batch_of_40_all_scores_equal():
+    ctx = tuple(2000 + (211 * i) % 900 for i in range(40))
+    spec = W.small_decode_spec(batch=40, context=ctx, capacity=3000, topk=64, steps=1, seed=25)
+    _decode_session(spec, check_seqs=[3, 38], steps=1, step_fn=_zero_w, exact_sel=True)
+
+
+@pytest.mark.slow
+def test_decode_batch_of_32_candidate_overflow():
+    # rows of more than 16,384 blocks with all scores equal, in a batch of 32: the threshold
+    # bin overflows the candidate buffer and the finish kernel takes the full-row select
+    ctx = tuple(66000 + 7 * i for i in range(32))
+    spec = W.small_decode_spec(batch=32, context=ctx, capacity=66400, topk=512, steps=1, seed=26)
+    _decode_session(spec, check_seqs=[0, 31], steps=1, step_fn=_zero_w, exact_sel=True,
+                    device_gen=True)
