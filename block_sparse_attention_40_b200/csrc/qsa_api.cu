@@ -295,6 +295,26 @@ qsa_status run_scores_and_topk(const void* q_idx, const void* w, const void* kba
   return QSA_OK;
 }
 
+// The attention kernel sets per-warpgroup register budgets at run time.  Before its first
+// launch, check that its register count per thread covers both budgets (a budget raise that
+// the launch cannot supply would wait forever), and set its shared-memory size.
+qsa_status prepare_attention() {
+  static std::atomic<int> ready{0};   // 1: checked and usable, 2: refused
+  int r = ready.load();
+  if (r == 0) {
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, k_sparse_attn) != cudaSuccess) return QSA_ERR_CUDA;
+    r = (static_cast<int64_t>(fa.numRegs) * AttnCfg::kThreads >= AttnCfg::kRegsNeeded) ? 1 : 2;
+    if (r == 2)
+      fprintf(stderr, "qsa: attention kernel built with %d registers per thread; %d needed\n",
+              fa.numRegs, (AttnCfg::kRegsNeeded + AttnCfg::kThreads - 1) / AttnCfg::kThreads);
+    ready.store(r);
+  }
+  if (r != 1) return QSA_ERR_UNSUPPORTED;
+  if (!set_smem(k_sparse_attn, AttnCfg::kSmemBytes)) return QSA_ERR_CUDA;
+  return QSA_OK;
+}
+
 qsa_status run_attention(const void* q, const void* k, const void* v, const int32_t* idx,
                          const int32_t* cnt, int num_seqs, const PrefillGeom& g,
                          unsigned char* ws, void* out, cudaStream_t s) {
@@ -324,7 +344,10 @@ qsa_status run_attention(const void* q, const void* k, const void* v, const int3
     if (!make_tmap(&maps.k[j], k, 2, dims, strides, box)) return QSA_ERR_CUDA;
     if (!make_tmap(&maps.v[j], v, 2, dims, strides, box)) return QSA_ERR_CUDA;
   }
-  if (!set_smem(k_sparse_attn, AttnCfg::kSmemBytes)) return QSA_ERR_CUDA;
+  {
+    const qsa_status pst = prepare_attention();
+    if (pst != QSA_OK) return pst;
+  }
   AttnArgs a{};
   a.oob_row = static_cast<int32_t>(g.T);
   a.plan = plan;
@@ -785,7 +808,10 @@ qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, 
       if (!make_tmap(&maps.k[j], cache->k_blocks, 2, dkv, skv, bkv)) return QSA_ERR_CUDA;
       if (!make_tmap(&maps.v[j], cache->v_blocks, 2, dkv, skv, bkv)) return QSA_ERR_CUDA;
     }
-    if (!set_smem(k_sparse_attn, AttnCfg::kSmemBytes)) return QSA_ERR_CUDA;
+    {
+    const qsa_status pst = prepare_attention();
+    if (pst != QSA_OK) return pst;
+  }
     AttnArgs a{};
     if (static_cast<uint64_t>(g.B) * 2 * g.cap >= 0x7fffffffull) return QSA_ERR_UNSUPPORTED;
     a.oob_row = static_cast<int32_t>(static_cast<int64_t>(g.B) * 2 * g.cap);

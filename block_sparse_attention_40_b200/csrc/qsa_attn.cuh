@@ -16,11 +16,16 @@
 //   O += P V         tcgen05, A = P (TMEM), B = V chunk (smem, MN-major), D = O in TMEM;
 //                    its completion frees the V slot
 // K/V rows are gathered with TMA boxes of 4..128 rows x 64 dims, one per naturally aligned
-// power-of-two piece of each run of consecutive blocks (no multicast).
+// power-of-two piece of each run of consecutive blocks (no multicast).  The boxes of a chunk
+// are spread over several producer warps (3 for K, 4 for V): on this part the rate at which a
+// warp's TMA copies go out is what limits a gather of small boxes, and it adds up over warps.
 //
-// Warp roles: warps 0-7 softmax (warp w owns TMEM lanes 32(w%4)..+31; warps 0-3 handle keys
-// 0-63 of each chunk, warps 4-7 keys 64-127), warp 8 Q+K producer, warp 9 V producer,
-// warp 10 TMEM allocation + MMA issue.
+// Warp roles (512 threads): warps 0-7 softmax (warp w owns TMEM lanes 32(w%4)..+31; warps 0-3
+// handle keys 0-63 of each chunk, warps 4-7 keys 64-127), warp 8 TMEM allocation + MMA issue,
+// warps 9-11 K producers (warp 9 also loads Q), warps 12-15 V producers.  The softmax
+// warpgroups raise their register budget to kRegsSoftmax, the other two lower theirs to
+// kRegsOther (setmaxnreg); the host checks before the first launch that the launch's
+// registers cover both.
 #pragma once
 
 #include "qsa_common.cuh"
@@ -29,7 +34,14 @@
 namespace qsa {
 
 struct AttnCfg {
-  static constexpr int kThreads = 352;   // 8 softmax warps, K and V producers, MMA
+  static constexpr int kThreads = 512;   // 8 softmax warps, MMA, 3 K and 4 V producers
+  static constexpr int kMmaWarp = 8;
+  static constexpr int kKWarp0 = 9, kKWarps = 3;
+  static constexpr int kVWarp0 = 12, kVWarps = 4;
+  static constexpr int kRegsSoftmax = 168;
+  static constexpr int kRegsOther = 80;
+  // registers the launch must provide for the two budgets above (checked on the host)
+  static constexpr int kRegsNeeded = 256 * kRegsSoftmax + 256 * kRegsOther;
   static constexpr int kChunkBlocks = 32;
   static constexpr int kChunkKeys = 128;
   static constexpr int kQBytes = 128 * kHeadDim * 2;         // 32 KB (2 panels of 16 KB)
@@ -97,16 +109,18 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// Producer of one operand stream (K or V) of a tile.  Lane u of the warp owns union slot u of
-// the chunk.  Maximal runs of consecutive block ids (and the run of padding slots past the
-// end of the union) are cut into power-of-two pieces; the first lane of each run issues one
-// TMA box per piece (rows 4*blk.., two 64-dim panels).  Padding rows come from an
-// out-of-range coordinate and are zero-filled.
+// Producer of one operand stream (K or V) of a tile, run by nw warps (this one is number w).
+// Lane u of each warp owns union slot u of the chunk.  Maximal runs of consecutive block ids
+// (and the run of padding slots past the end of the union) are cut into power-of-two pieces;
+// the first lane of each run issues one TMA box per piece (rows 4*blk.., two 64-dim panels).
+// Run r of a chunk (in slot order) goes to warp r mod nw; warp 0 posts the chunk's bytes.
+// Padding rows come from an out-of-range coordinate and are zero-filled.
 __device__ __forceinline__ void attn_producer(const CUtensorMap* maps, unsigned char* ring,
                                               uint64_t* full, uint64_t* empty, int stages,
                                               const int32_t* uni, int U, int c_begin, int nchunks,
                                               int64_t kv_row_base, int col0, int32_t oob_row,
-                                              volatile int* abort, DevStatus st, uint32_t site) {
+                                              int w, int nw, volatile int* abort, DevStatus st,
+                                              uint32_t site) {
   const int lane = threadIdx.x & 31;
   int upos = c_begin * AttnCfg::kChunkBlocks + lane;
   int blk_next = upos < U ? uni[upos] : -1;
@@ -120,12 +134,14 @@ __device__ __forceinline__ void attn_producer(const CUtensorMap* maps, unsigned 
     if (lane == 0) ok = mbar_wait(&empty[s], ((i / stages) & 1) ^ 1, abort, st, site);
     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
     if (!ok) break;
-    if (lane == 0) mbar_arrive_expect_tx(&full[s], AttnCfg::kKVBytes);
+    if (lane == 0 && w == 0) mbar_arrive_expect_tx(&full[s], AttnCfg::kKVBytes);
     __syncwarp();
     const int prev = __shfl_up_sync(0xffffffffu, blk, 1);
     const bool start = lane == 0 || (blk < 0) != (prev < 0) || (blk >= 0 && blk != prev + 1);
     const unsigned starts = __ballot_sync(0xffffffffu, start);
-    if (start) {
+    // (a box may complete before warp 0 posts the bytes: the phase cannot end while the
+    // posting arrival is missing)
+    if (start && __popc(starts & ((1u << lane) - 1u)) % nw == w) {
       const unsigned later = starts & ~((2u << lane) - 1u);   // run starts after this lane
       const int run_end = later ? __ffs(later) - 1 : 32;
       int off = 0;
@@ -262,7 +278,7 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
     }
     fence_proxy_async_smem();
   }
-  if (warp == 10) {
+  if (warp == C::kMmaWarp) {
     tmem_alloc(s_tmem, C::kTmemCols);
     tmem_relinquish();
   }
@@ -277,9 +293,13 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
   const int mwords = args.pl.umax / 32;
   const int col0 = args.decode ? 0 : g * kHeadDim;
 
-  if (warp == 8) {
-    // ---------------- Q + K producer ----------------
-    if (lane == 0) {
+  if (warp >= 8) {
+  // warpgroups 2 and 3 (MMA and producers) give registers up for the softmax warpgroups
+  regs_lower<C::kRegsOther>();
+  if (warp >= C::kKWarp0 && warp < C::kKWarp0 + C::kKWarps) {
+    // ---------------- Q + K producers ----------------
+    const int kw = warp - C::kKWarp0;
+    if (kw == 0 && lane == 0) {
       prefetch_tmap(&maps.q);
       for (int j = 0; j < kNumBoxSizes; ++j) prefetch_tmap(&maps.k[j]);
       const uint32_t qbytes = 2u * kGroup * R * 128u;   // full box, out-of-range rows zero-filled
@@ -290,17 +310,18 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
     }
     __syncwarp();
     attn_producer(maps.k, sK, k_full, k_empty, C::kKStages, uni, U, c_begin, nchunks,
-                  kv_row_base, col0, args.oob_row, s_abort, args.st, 20);
-    if (lane == 0 && *s_abort) mbar_drain(q_full, 0);
-  } else if (warp == 9) {
-    // ---------------- V producer ----------------
-    if (lane == 0)
+                  kv_row_base, col0, args.oob_row, kw, C::kKWarps, s_abort, args.st, 20);
+    if (kw == 0 && lane == 0 && *s_abort) mbar_drain(q_full, 0);
+  } else if (warp >= C::kVWarp0) {
+    // ---------------- V producers ----------------
+    const int vw = warp - C::kVWarp0;
+    if (vw == 0 && lane == 0)
       for (int j = 0; j < kNumBoxSizes; ++j) prefetch_tmap(&maps.v[j]);
     __syncwarp();
     attn_producer(maps.v, sV, v_full, v_empty, C::kVStages, uni, U, c_begin, nchunks,
-                  kv_row_base, col0, args.oob_row, s_abort, args.st, 27);
-  } else if (warp == 10) {
-    // ---------------- MMA issuer ----------------
+                  kv_row_base, col0, args.oob_row, vw, C::kVWarps, s_abort, args.st, 27);
+  } else {
+    // ---------------- MMA issuer (warp kMmaWarp) ----------------
     if (lane == 0) {
       const uint32_t sQ0 = smem_u32(sQ);
       bool ok = mbar_wait(q_full, 0, s_abort, args.st, 21);
@@ -346,7 +367,9 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
       umma_commit(mma_done);
       mbar_drain(mma_done, 0);
     }
+  }
   } else {
+    regs_raise<C::kRegsSoftmax>();
     // ---------------- softmax (warps 0-7) ----------------
     // Two warpgroups share each row: warpgroup wg handles keys [64 wg, 64 wg + 64) of every
     // chunk and dims [64 wg, 64 wg + 64) of O.  Row maxima are exchanged through shared memory
@@ -518,7 +541,7 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 10) {
+  if (warp == C::kMmaWarp) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);

@@ -147,6 +147,16 @@ __device__ __forceinline__ void named_barrier_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// ---- per-warpgroup register budgets (all four warps of a warpgroup execute these) ---------
+template <int N>
+__device__ __forceinline__ void regs_raise() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_lower() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---- programmatic dependent launch -------------------------------------------------------
 // A kernel launched with programmatic stream serialization may start while the kernel before
 // it in the stream is still running.  pdl_wait blocks until that kernel has completed and its
