@@ -291,14 +291,7 @@ __global__ void __launch_bounds__(ScoreCfg<NTOK>::kThreads, ScoreCfg<NTOK>::kCta
         const bool valid = tok < wk.ntok && blk < pos / kBlock;
         if (valid) args.scores[(wk.out_row0 + tok) * args.ld + blk] = s;
         if constexpr (NTOK == 1) {
-          if (args.hist) {
-            const unsigned act = __ballot_sync(0xffffffffu, valid);
-            if (valid) {
-              const uint32_t bin = float_key(s) >> 20;
-              const unsigned peers = __match_any_sync(act, bin);
-              if (lane == __ffs(peers) - 1) atomicAdd(&sHist[bin], static_cast<uint32_t>(__popc(peers)));
-            }
-          }
+          if (args.hist && valid) atomicAdd(&sHist[float_key(s) >> 20], 1u);
         }
       }
     }
