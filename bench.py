@@ -232,14 +232,35 @@ def run_qsa(args, rank, world, local):
             reset_cache()
             flush()
             ev["d0"].record(stream)
-            cache.append(st["k"], st["v"], st["k_idx"])
-            dec.run(st["q"], st["q_idx"], st["w"], out=dec_out)
+            if dec_graph is not None:
+                dec_graph.replay()
+            else:
+                cache.append(st["k"], st["v"], st["k_idx"])
+                dec.run(st["q"], st["q_idx"], st["w"], out=dec_out)
             ev["d1"].record(stream)
 
     names = ["p0", "p1", "p2", "d0", "d1"]
+    dec_graph = None
+    graph_launches = 0
     for _ in range(args.warmup):
         step(False, {n: torch.cuda.Event(enable_timing=True) for n in names})
     torch.cuda.synchronize(dev)
+    if do_decode and args.graph:
+        # one decode step (append + decode) captured as a CUDA graph and replayed per step;
+        # the cache is reset outside the graph, so every replay sees the same state
+        reset_cache()
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        n0 = B.launch_count()
+        with torch.cuda.graph(g):
+            cache.append(st["k"], st["v"], st["k_idx"])
+            dec.run(st["q"], st["q_idx"], st["w"], out=dec_out)
+        torch.cuda.synchronize(dev)
+        graph_launches = B.launch_count() - n0   # kernels each replay runs
+        dec_graph = g
+        for _ in range(args.warmup):
+            step(False, {n: torch.cuda.Event(enable_timing=True) for n in names})
+        torch.cuda.synchronize(dev)
     barrier(world)
     launches0 = B.launch_count()
     evs = [{n: torch.cuda.Event(enable_timing=True) for n in names} for _ in range(args.steps)]
@@ -253,7 +274,7 @@ def run_qsa(args, rank, world, local):
     torch.cuda.synchronize(dev)
     barrier(world)
     clk = clocks.stop()
-    launches = B.launch_count() - launches0
+    launches = B.launch_count() - launches0 + args.steps * graph_launches
     sel_ms = sum(e["p0"].elapsed_time(e["p1"]) for e in evs) if do_prefill else 0.0
     att_ms = sum(e["p1"].elapsed_time(e["p2"]) for e in evs) if do_prefill else 0.0
     dec_ms = sum(e["d0"].elapsed_time(e["d1"]) for e in evs) if do_decode else 0.0
@@ -323,6 +344,7 @@ def run_qsa(args, rank, world, local):
                do_decode=do_decode)
     if do_decode:
         res["dec_bytes"] = sum(decode_bytes_per_seq(L + 1) for L in spec.context)
+        res["dec_timing"] = "cuda graph replay of append + decode" if dec_graph is not None else "eager launches"
     return res
 
 
@@ -388,6 +410,8 @@ def main():
     ap.add_argument("--prefill-len", type=int, default=PREFILL_T,
                     help="prefill sequence length (default 65536; smaller only for profiling)")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--no-graph", dest="graph", action="store_false",
+                    help="time the decode step as eager launches instead of a CUDA graph replay")
     ap.add_argument("--no-cpu-baseline", dest="cpu", action="store_false")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -425,6 +449,7 @@ def main():
         dms = r["dec_ms"] / K
         gbs = r["dec_bytes"] / (dms / 1e3) / 1e9
         dec = {"value": world * args.decode_batch / (dms / 1e3), "unit": "tokens/s", "ms_per_step": dms,
+               "timing": r["dec_timing"],
                "roofline": {"kernel": "whole decode step (append, indexer, top-k, plan, "
                                       "attention, combine)", "bound": "hbm", "achieved": gbs,
                             "peak": peaks["hbm_gbs"], "unit": "GB/s",
