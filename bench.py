@@ -436,7 +436,12 @@ def main():
                             "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
                             "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
                             "peak_source": f"{r['peak_src']} bf16 burst",
-                            "traffic": None,
+                            # dram__bytes_read + dram__bytes_write of this kernel from one ncu
+                            # capture of the 32K prefill (profiles/k_sparse_attn_prefill_32k.md),
+                            # scaled by tokens (the traffic is q, the plan and the output; K/V
+                            # stay in L2)
+                            "traffic": 491.918e6 * args.prefill_len / 32768,
+                            "traffic_source": "ncu capture at 32K, scaled by tokens",
                             "algorithmic": f"{attn_flops / 1e12:.4f} TFLOP selected-token per launch"}
         idx_flops = prefill_indexer_flops(args.prefill_len)
         line["prefill"] = {"tokens_per_s": world * args.prefill_len / (pre_ms / 1e3),
