@@ -29,7 +29,7 @@ struct ScoreCfg {
   static constexpr int kTmemCols = kAccCols * kNumAcc;    // 512 / 128
   static constexpr int kStages = NTOK == 16 ? 4 : 5;     // decode: 2 CTAs per SM
   static constexpr int kCtasPerSm = NTOK == 16 ? 1 : 2;
-  static constexpr int kEpiWarps = NTOK == 16 ? 8 : 4;
+  static constexpr int kEpiWarps = NTOK == 16 ? 16 : 4;   // prefill: 4 token groups x 4 lane quarters
   static constexpr int kThreads = 64 + 32 * kEpiWarps;
   static constexpr int kABytes = 128 * kIdxDim * 2;       // 16 KB
   static constexpr int kBBytes = kN * kIdxDim * 2;        // 32 KB / 2 KB
@@ -261,8 +261,8 @@ __global__ void __launch_bounds__(ScoreCfg<NTOK>::kThreads, ScoreCfg<NTOK>::kCta
     // ---------------- epilogue ----------------
     const int ew = warp - 2;
     const int quarter = warp & 3;          // TMEM lanes this warp may access
-    const int part = ew / 4;               // which half of the tokens (prefill)
-    constexpr int kTokPerWarp = NTOK == 16 ? 8 : 1;
+    const int part = ew / 4;               // which group of four tokens (prefill)
+    constexpr int kTokPerWarp = NTOK == 16 ? 4 : 1;
     const int tok_base = part * kTokPerWarp;
     for (int i = 0; i < wk.n_mtiles; ++i) {
       const int a = i % C::kNumAcc;
@@ -274,7 +274,7 @@ __global__ void __launch_bounds__(ScoreCfg<NTOK>::kThreads, ScoreCfg<NTOK>::kCta
       uint32_t acc[kTokPerWarp * kIdxHeads];
       if constexpr (NTOK == 16) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tbase + 32 * c, acc + 32 * c);
+        for (int c = 0; c < kTokPerWarp / 2; ++c) tmem_ld32(tbase + 32 * c, acc + 32 * c);
       } else {
         tmem_ld16(tbase, acc);
       }
