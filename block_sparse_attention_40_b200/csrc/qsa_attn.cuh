@@ -20,12 +20,12 @@
 // are spread over several producer warps (3 for K, 4 for V): on this part the rate at which a
 // warp's TMA copies go out is what limits a gather of small boxes, and it adds up over warps.
 //
-// Warp roles (512 threads): warps 0-7 softmax (warp w owns TMEM lanes 32(w%4)..+31; warps 0-3
-// handle keys 0-63 of each chunk, warps 4-7 keys 64-127), warp 8 TMEM allocation + MMA issue,
-// warps 9-11 K producers (warp 9 also loads Q), warps 12-15 V producers.  The softmax
-// warpgroups raise their register budget to kRegsSoftmax, the other two lower theirs to
-// kRegsOther (setmaxnreg); the host checks before the first launch that the launch's
-// registers cover both.
+// Warp roles (kSoftGroups = 2: 512 threads): warps 0-7 softmax (warp w owns TMEM lanes
+// 32(w%4)..+31; warpgroup g handles keys 64g..64g+63 of each chunk), warp 8 TMEM allocation +
+// MMA issue, warps 9-11 K producers (warp 9 also loads Q), warps 12-15 V producers.  The
+// softmax warpgroups raise their register budget to kRegsSoftmax, the other two lower theirs
+// to kRegsOther (setmaxnreg); the host checks before the first launch that the launch's
+// registers cover both.  Four softmax warpgroups (32 keys each, 768 threads) measured slower.
 #pragma once
 
 #include "qsa_common.cuh"
@@ -33,15 +33,20 @@
 
 namespace qsa {
 
+#ifndef QSA_ATTN_SOFT_GROUPS
+#define QSA_ATTN_SOFT_GROUPS 2
+#endif
 struct AttnCfg {
-  static constexpr int kThreads = 512;   // 8 softmax warps, MMA, 3 K and 4 V producers
-  static constexpr int kMmaWarp = 8;
-  static constexpr int kKWarp0 = 9, kKWarps = 3;
-  static constexpr int kVWarp0 = 12, kVWarps = 4;
-  static constexpr int kRegsSoftmax = 168;
-  static constexpr int kRegsOther = 80;
+  static constexpr int kSoftGroups = QSA_ATTN_SOFT_GROUPS;   // softmax warpgroups (2 or 4)
+  static constexpr int kSoftWarps = 4 * kSoftGroups;
+  static constexpr int kMmaWarp = kSoftWarps;
+  static constexpr int kKWarp0 = kSoftWarps + 1, kKWarps = 3;
+  static constexpr int kVWarp0 = kSoftWarps + 4, kVWarps = 4;
+  static constexpr int kThreads = 32 * (kSoftWarps + 8);   // + MMA, 3 K and 4 V producers
+  static constexpr int kRegsSoftmax = kSoftGroups == 2 ? 168 : 96;
+  static constexpr int kRegsOther = kSoftGroups == 2 ? 80 : 48;
   // registers the launch must provide for the two budgets above (checked on the host)
-  static constexpr int kRegsNeeded = 256 * kRegsSoftmax + 256 * kRegsOther;
+  static constexpr int kRegsNeeded = 128 * kSoftGroups * kRegsSoftmax + 256 * kRegsOther;
   static constexpr int kChunkBlocks = 32;
   static constexpr int kChunkKeys = 128;
   static constexpr int kQBytes = 128 * kHeadDim * 2;         // 32 KB (2 panels of 16 KB)
@@ -52,7 +57,7 @@ struct AttnCfg {
   static constexpr int kKOff = kQBytes;
   static constexpr int kVOff = kKOff + kKStages * kKVBytes;
   static constexpr int kXOff = kVOff + kVStages * kKVBytes;    // row-max / row-sum exchange
-  static constexpr int kXBytes = (2 * 2 * 128 + 2 * 128) * 4;
+  static constexpr int kXBytes = (2 * kSoftGroups * 128 + kSoftGroups * 128) * 4;
   static constexpr int kBarOff = kXOff + kXBytes;
   static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 1 + 1 + 1;
   static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
@@ -180,8 +185,8 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
   unsigned char* sQ = smem + C::kQOff;
   unsigned char* sK = smem + C::kKOff;
   unsigned char* sV = smem + C::kVOff;
-  float* xmax = reinterpret_cast<float*>(smem + C::kXOff);   // [parity][wg][128]
-  float* xsum = xmax + 2 * 2 * 128;                           // [wg][128]
+  float* xmax = reinterpret_cast<float*>(smem + C::kXOff);   // [parity][group][128]
+  float* xsum = xmax + 2 * C::kSoftGroups * 128;              // [group][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
@@ -258,7 +263,7 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 8);
+      mbar_init(&p_full[i], C::kSoftWarps);
       mbar_init(&p_free[i], 1);
     }
     mbar_init(pv_done, 1);
@@ -293,8 +298,8 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
   const int mwords = args.pl.umax / 32;
   const int col0 = args.decode ? 0 : g * kHeadDim;
 
-  if (warp >= 8) {
-  // warpgroups 2 and 3 (MMA and producers) give registers up for the softmax warpgroups
+  if (warp >= C::kSoftWarps) {
+  // the last two warpgroups (MMA and producers) give registers up for the softmax warpgroups
   regs_lower<C::kRegsOther>();
   if (warp >= C::kKWarp0 && warp < C::kKWarp0 + C::kKWarps) {
     // ---------------- Q + K producers ----------------
@@ -370,11 +375,14 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
   }
   } else {
     regs_raise<C::kRegsSoftmax>();
-    // ---------------- softmax (warps 0-7) ----------------
-    // Two warpgroups share each row: warpgroup wg handles keys [64 wg, 64 wg + 64) of every
-    // chunk and dims [64 wg, 64 wg + 64) of O.  Row maxima are exchanged through shared memory
-    // (double-buffered by chunk parity, one named barrier per chunk); partial row sums are
-    // combined once at the end.  Both halves take identical rescale decisions.
+    // ---------------- softmax (warps 0 .. 4 kSoftGroups - 1) ----------------
+    // kSoftGroups warpgroups share each row: group sg handles keys [kCols sg, kCols (sg + 1))
+    // of every chunk and dims [kCols sg, ...) of O.  Row maxima are exchanged through shared
+    // memory (double-buffered by chunk parity, one named barrier per chunk); partial row sums
+    // are combined once at the end.  All groups take identical rescale decisions.
+    constexpr int kSG = C::kSoftGroups;
+    constexpr int kCols = 128 / kSG;              // keys (and O dims) per group
+    constexpr int kBlk = kCols / kBlock;          // blocks per group
     const int wg = warp >> 2;
     const int quarter = warp & 3;           // TMEM lanes 32q .. 32q+31
     const int row = quarter * 32 + lane;
@@ -395,31 +403,31 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
     for (int i = 0; i < nchunks; ++i) {
       const int b = i & 1;
       const int q = c_begin + i;
-      const uint32_t mword = (mword_next >> (16 * wg)) & 0xffffu;   // my 16 blocks
+      const uint32_t mword = (mword_next >> (kBlk * wg)) & ((1u << kBlk) - 1u);   // my blocks
       if (row_ok && i + 1 < nchunks) mword_next = mrow[q + 1];
       bool got = ok ? mbar_wait(&s_full[b], (i >> 1) & 1, s_abort, args.st, 24) : false;
       if (__any_sync(0xffffffffu, !got)) ok = false;   // also reconverges the warp
       tc_fence_after();
-      uint32_t sv[64];
+      uint32_t sv[kCols];
       const uint32_t ts = tmem + lane_base + b * 128;
       float mx = -INFINITY;
       if (ok && warp_active) {
-        tmem_ld32(ts + 64 * wg, sv);
-        tmem_ld32(ts + 64 * wg + 32, sv + 32);
+#pragma unroll
+        for (int c = 0; c < kCols / 32; ++c) tmem_ld32(ts + kCols * wg + 32 * c, sv + 32 * c);
         tmem_wait_ld();
         // keys of blocks this row's token did not select -> -inf
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
+        for (int u = 0; u < kBlk; ++u) {
           const float bias = ((mword >> u) & 1u) ? 0.f : -INFINITY;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             sv[4 * u + kk] = __float_as_uint(__uint_as_float(sv[4 * u + kk]) + bias);
         }
         // the own block: hide the tokens after the query (only where it lies)
-        const int tu = tail_u - q * C::kChunkBlocks - 16 * wg;
-        if (__any_sync(0xffffffffu, tu >= 0 && tu < 16)) {
+        const int tu = tail_u - q * C::kChunkBlocks - kBlk * wg;
+        if (__any_sync(0xffffffffu, tu >= 0 && tu < kBlk)) {
 #pragma unroll
-          for (int u = 0; u < 16; ++u) {
+          for (int u = 0; u < kBlk; ++u) {
             if (u == tu) {
               if (tail_last < 1) sv[4 * u + 1] = __float_as_uint(-INFINITY);
               if (tail_last < 2) sv[4 * u + 2] = __float_as_uint(-INFINITY);
@@ -431,17 +439,18 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
 #pragma unroll
         for (int j = 0; j < 8; ++j) mxs[j] = __uint_as_float(sv[j]);
 #pragma unroll
-        for (int j = 8; j < 64; ++j) mxs[j & 7] = fmaxf(mxs[j & 7], __uint_as_float(sv[j]));
+        for (int j = 8; j < kCols; ++j) mxs[j & 7] = fmaxf(mxs[j & 7], __uint_as_float(sv[j]));
         mx = fmaxf(fmaxf(fmaxf(mxs[0], mxs[1]), fmaxf(mxs[2], mxs[3])),
                    fmaxf(fmaxf(mxs[4], mxs[5]), fmaxf(mxs[6], mxs[7])));
       }
-      // exchange the half-row maxima (every softmax warp takes part, active or not)
-      xmax[(b * 2 + wg) * 128 + row] = mx;
+      // exchange the partial row maxima (every softmax warp takes part, active or not)
+      xmax[(b * kSG + wg) * 128 + row] = mx;
       tc_fence_before();
-      named_barrier_sync(1, 256);
+      named_barrier_sync(1, 128 * kSG);
       tc_fence_after();
       if (ok && warp_active) {
-        mx = fmaxf(mx, xmax[(b * 2 + (wg ^ 1)) * 128 + row]);
+#pragma unroll
+        for (int o = 1; o < kSG; ++o) mx = fmaxf(mx, xmax[(b * kSG + ((wg + o) % kSG)) * 128 + row]);
         const float m_cand = fmaxf(m, mx * sl2);
         const bool need = m_cand > m + 8.f || (m == -INFINITY && m_cand > -INFINITY);
         const bool rescale = __any_sync(0xffffffffu, need);
@@ -455,27 +464,31 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
         // consumed at pair j/2 <= j
         float lsum[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
+        for (int j = 0; j < kCols / 2; ++j) {
           const float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * j]), sl2, mneg));
           const float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * j + 1]), sl2, mneg));
           lsum[j & 3] += p0 + p1;
           sv[j] = pack_bf16x2(p0, p1);
         }
         l = l * alpha + ((lsum[0] + lsum[1]) + (lsum[2] + lsum[3]));
-        // packed P of keys 64 wg .. 64 wg + 63 -> columns 32 wg .. 32 wg + 31 of the buffer
-        // (the other half's S there was loaded before the barrier above)
-        tmem_st32(ts + 32 * wg, sv);
+        // packed P of my keys -> columns kCols/2 sg .. of the buffer (every group's S there was
+        // loaded before the barrier above)
+        if constexpr (kCols == 64) {
+          tmem_st32(ts + 32 * wg, sv);
+        } else {
+          tmem_st16(ts + 16 * wg, sv);
+        }
         tmem_wait_st();
         if (rescale && i > 0) {
           // O holds P.V of chunks < i-1 and maybe i-1: wait until chunk i-1 is in, rescale
-          // my half of O.  P.V of chunk i cannot start before this warp arrives on p_full.
+          // my dims of O.  P.V of chunk i cannot start before this warp arrives on p_full.
           const bool gotpv = mbar_wait(pv_done, (i - 1) & 1, s_abort, args.st, 25);
           if (__any_sync(0xffffffffu, !gotpv)) ok = false;
           if (ok) {
             tc_fence_after();
-            const uint32_t to = tmem_O + lane_base + 64 * wg;
+            const uint32_t to = tmem_O + lane_base + kCols * wg;
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            for (int c = 0; c < kCols / 32; ++c) {
               uint32_t ov[32];
               tmem_ld32(to + 32 * c, ov);
               tmem_wait_ld();
@@ -491,10 +504,12 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[b]);
     }
-    // combine the half-row sums
+    // combine the partial row sums
     xsum[wg * 128 + row] = l;
-    named_barrier_sync(1, 256);
-    const float l_all = l + xsum[(wg ^ 1) * 128 + row];
+    named_barrier_sync(1, 128 * kSG);
+    float l_all = 0.f;
+#pragma unroll
+    for (int o = 0; o < kSG; ++o) l_all += xsum[o * 128 + row];
     if (ok && nchunks > 0) {
       // a dedicated barrier: two P.V may still be in flight here, so a parity wait on
       // pv_done could match an older phase
@@ -502,18 +517,18 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
       if (!__any_sync(0xffffffffu, !got)) {
         tc_fence_after();
         if (warp_active) {
-          const uint32_t to = tmem_O + lane_base + 64 * wg;
-          uint32_t ov[64];
-          tmem_ld32(to, ov);
-          tmem_ld32(to + 32, ov + 32);
+          const uint32_t to = tmem_O + lane_base + kCols * wg;
+          uint32_t ov[kCols];
+#pragma unroll
+          for (int c = 0; c < kCols / 32; ++c) tmem_ld32(to + 32 * c, ov + 32 * c);
           tmem_wait_ld();
           if (row_ok) {
             if (!args.decode || args.splits == 1) {   // one split: the final output directly
               const float inv = l_all > 0.f ? 1.f / l_all : 0.f;
               __nv_bfloat16* o = args.out + ((tok_row0 + tr) * kHeads + g * kGroup + hr) * kHeadDim +
-                                 64 * wg;
+                                 kCols * wg;
 #pragma unroll
-              for (int c = 0; c < 8; ++c) {
+              for (int c = 0; c < kCols / 8; ++c) {
                 uint4 v;
                 v.x = pack_bf16x2(__uint_as_float(ov[8 * c + 0]) * inv, __uint_as_float(ov[8 * c + 1]) * inv);
                 v.y = pack_bf16x2(__uint_as_float(ov[8 * c + 2]) * inv, __uint_as_float(ov[8 * c + 3]) * inv);
@@ -528,9 +543,9 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
                 args.part_m[pr] = m;
                 args.part_l[pr] = l_all;
               }
-              float4* po = reinterpret_cast<float4*>(args.part_o + pr * kHeadDim + 64 * wg);
+              float4* po = reinterpret_cast<float4*>(args.part_o + pr * kHeadDim + kCols * wg);
 #pragma unroll
-              for (int c = 0; c < 16; ++c)
+              for (int c = 0; c < kCols / 4; ++c)
                 po[c] = make_float4(__uint_as_float(ov[4 * c]), __uint_as_float(ov[4 * c + 1]),
                                     __uint_as_float(ov[4 * c + 2]), __uint_as_float(ov[4 * c + 3]));
             }
