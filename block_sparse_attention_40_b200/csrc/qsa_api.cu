@@ -302,16 +302,22 @@ qsa_status prepare_attention() {
   static std::atomic<int> ready{0};   // 1: checked and usable, 2: refused
   int r = ready.load();
   if (r == 0) {
-    cudaFuncAttributes fa{};
-    if (cudaFuncGetAttributes(&fa, k_sparse_attn) != cudaSuccess) return QSA_ERR_CUDA;
-    r = (static_cast<int64_t>(fa.numRegs) * AttnCfg::kThreads >= AttnCfg::kRegsNeeded) ? 1 : 2;
-    if (r == 2)
-      fprintf(stderr, "qsa: attention kernel built with %d registers per thread; %d needed\n",
-              fa.numRegs, (AttnCfg::kRegsNeeded + AttnCfg::kThreads - 1) / AttnCfg::kThreads);
+    r = 1;
+    for (const void* fn : {reinterpret_cast<const void*>(k_sparse_attn<false>),
+                           reinterpret_cast<const void*>(k_sparse_attn<true>)}) {
+      cudaFuncAttributes fa{};
+      if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) return QSA_ERR_CUDA;
+      if (static_cast<int64_t>(fa.numRegs) * AttnCfg::kThreads < AttnCfg::kRegsNeeded) {
+        fprintf(stderr, "qsa: attention kernel built with %d registers per thread; %d needed\n",
+                fa.numRegs, (AttnCfg::kRegsNeeded + AttnCfg::kThreads - 1) / AttnCfg::kThreads);
+        r = 2;
+      }
+    }
     ready.store(r);
   }
   if (r != 1) return QSA_ERR_UNSUPPORTED;
-  if (!set_smem(k_sparse_attn, AttnCfg::kSmemBytes)) return QSA_ERR_CUDA;
+  if (!set_smem(k_sparse_attn<false>, AttnCfg::kSmemBytes)) return QSA_ERR_CUDA;
+  if (!set_smem(k_sparse_attn<true>, AttnCfg::kSmemBytes)) return QSA_ERR_CUDA;
   return QSA_OK;
 }
 
@@ -359,7 +365,7 @@ qsa_status run_attention(const void* q, const void* k, const void* v, const int3
   a.out = reinterpret_cast<__nv_bfloat16*>(out);
   a.st = dev_status(ws);
   dim3 grid(g.attn_tiles, 2, 1);
-  k_sparse_attn<<<grid, AttnCfg::kThreads, AttnCfg::kSmemBytes, s>>>(maps, a);
+  k_sparse_attn<false><<<grid, AttnCfg::kThreads, AttnCfg::kSmemBytes, s>>>(maps, a);
   QSA_CHECK_LAUNCH();
   return QSA_OK;
 }
@@ -826,7 +832,7 @@ qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, 
     a.st = dev_status(ws);
     dim3 grid(g.B, 2, g.splits);
     a.out = reinterpret_cast<__nv_bfloat16*>(out);   // written directly with one split
-    QSA_CHECK_PDL(launch_pdl(k_sparse_attn, grid, dim3(AttnCfg::kThreads), AttnCfg::kSmemBytes,
+    QSA_CHECK_PDL(launch_pdl(k_sparse_attn<true>, grid, dim3(AttnCfg::kThreads), AttnCfg::kSmemBytes,
                              s, maps, a));
     if (g.splits > 1) {
       const int warps = g.B * kHeads;

@@ -15,6 +15,11 @@
 //                    by more than 2^8); P = exp2(.) written back over S in TMEM as bf16
 //   O += P V         tcgen05, A = P (TMEM), B = V chunk (smem, MN-major), D = O in TMEM;
 //                    its completion frees the V slot
+// Decode (kDec, one query token, 12 valid rows): the 12 head rows are loaded into each of the
+// four TMEM lane quarters, and each copy takes a quarter of every chunk's keys with its own
+// running max and sum, so that all softmax warps share the work instead of one warp per group;
+// P then lives in its own TMEM columns and the four copies are merged at the end.
+//
 // K/V rows are gathered with TMA boxes of 4..128 rows x 64 dims, one per naturally aligned
 // power-of-two piece of each run of consecutive blocks (no multicast).  The boxes of a chunk
 // are spread over several producer warps (3 for K, 4 for V): on this part the rate at which a
@@ -176,6 +181,8 @@ __device__ __forceinline__ void attn_producer(const CUtensorMap* maps, unsigned 
   }
 }
 
+// kDec: decode layout (one query token per tile; see the decode softmax below).
+template <bool kDec>
 __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
     k_sparse_attn(const __grid_constant__ AttnMaps maps, AttnArgs args) {
   using C = AttnCfg;
@@ -213,7 +220,7 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
   const int R = args.pl.R;
   const int nchunks_all = (U + C::kChunkBlocks - 1) / C::kChunkBlocks;
   int c_begin = 0, c_end = nchunks_all;
-  if (args.decode) {
+  if (kDec) {
     const int per = (nchunks_all + args.splits - 1) / args.splits;
     c_begin = split * per;
     c_end = c_begin + per < nchunks_all ? c_begin + per : nchunks_all;
@@ -224,7 +231,7 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
   int64_t tok_row0 = 0;   // global token row (prefill) / sequence (decode) of token 0
   int pos0 = 0;           // position within the sequence of token 0
   int64_t kv_row_base = 0;
-  if (args.decode) {
+  if (kDec) {
     tok_row0 = tile;
     pos0 = rec[2];   // p = len - 1 of the sequence
     kv_row_base = (static_cast<int64_t>(tile) * 2 + g) * args.cap_blocks * kBlock;
@@ -241,7 +248,7 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
 
   if (nchunks == 0 || ntok == 0) {
     // decode split without keys: write an empty partial
-    if (args.decode && ntok > 0 && threadIdx.x < kGroup) {
+    if (kDec && ntok > 0 && threadIdx.x < kGroup) {
       const int64_t pr = ((static_cast<int64_t>(tile) * 2 + g) * args.splits + split) * kGroup +
                          threadIdx.x;
       args.part_m[pr] = -INFINITY;
@@ -272,12 +279,14 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
     *s_abort = 0;
     fence_mbar_init();
   }
-  // zero the rows of Q below the TMA box (rows 12R..127 are never written by TMA)
+  // zero the rows of Q that TMA never writes: rows 12R..127 (prefill), or rows 32q+12..32q+31
+  // of every lane quarter q (decode: the 12 head rows are loaded at rows 32q..32q+11)
   {
     const int box_rows = kGroup * R;
-    const int pad_rows = 128 - box_rows;
+    const int pad_rows = kDec ? 4 * (32 - kGroup) : 128 - box_rows;
     for (int i = threadIdx.x; i < pad_rows * 16; i += blockDim.x) {
-      const int r = box_rows + i / 16, c = i % 16;   // 16 x 16 B per row (both panels)
+      const int pr = i / 16, c = i % 16;   // 16 x 16 B per row (both panels)
+      const int r = kDec ? (pr / (32 - kGroup)) * 32 + kGroup + pr % (32 - kGroup) : box_rows + pr;
       const int panel = c / 8, cc = c % 8;
       *reinterpret_cast<uint4*>(sQ + panel * 16384 + r * 128 + cc * 16) = make_uint4(0, 0, 0, 0);
     }
@@ -296,7 +305,10 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
   const int32_t* uni = rec + args.pl.union_off();
   const uint32_t* masks = reinterpret_cast<const uint32_t*>(rec + args.pl.mask_off());
   const int mwords = args.pl.umax / 32;
-  const int col0 = args.decode ? 0 : g * kHeadDim;
+  const int col0 = kDec ? 0 : g * kHeadDim;
+  // P: written over S in prefill; in its own columns [384, 512) in decode
+  const uint32_t tmem_P = kDec ? tmem + 384 : tmem;
+  constexpr int kPStride = kDec ? 64 : 128;
 
   if (warp >= C::kSoftWarps) {
   // the last two warpgroups (MMA and producers) give registers up for the softmax warpgroups
@@ -308,10 +320,12 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
       prefetch_tmap(&maps.q);
       for (int j = 0; j < kNumBoxSizes; ++j) prefetch_tmap(&maps.k[j]);
       const uint32_t qbytes = 2u * kGroup * R * 128u;   // full box, out-of-range rows zero-filled
-      mbar_arrive_expect_tx(q_full, qbytes);
-      for (int half = 0; half < 2; ++half)
-        tma_load_3d(sQ + half * 16384, &maps.q, half * 64, g * kGroup,
-                    static_cast<int32_t>(tok_row0), q_full);
+      constexpr int kCopies = kDec ? 4 : 1;            // decode: one copy per lane quarter
+      mbar_arrive_expect_tx(q_full, kCopies * qbytes);
+      for (int cp = 0; cp < kCopies; ++cp)
+        for (int half = 0; half < 2; ++half)
+          tma_load_3d(sQ + half * 16384 + cp * 4096, &maps.q, half * 64, g * kGroup,
+                      static_cast<int32_t>(tok_row0), q_full);
     }
     __syncwarp();
     attn_producer(maps.k, sK, k_full, k_empty, C::kKStages, uni, U, c_begin, nchunks,
@@ -341,7 +355,8 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
         for (int k = 0; k < C::kChunkKeys / 16; ++k) {
           // B = V chunk, MN-major: 16 keys per step = 2048 bytes; next 64 dims at +16 KB
           const uint64_t db = smem_desc_sw128(sV0 + 2048 * k, 16384, 1024);
-          umma_ts(tmem_O, tmem + bj * 128 + 8 * k, db, C::kIdescPV, (j > 0 || k > 0) ? 1u : 0u);
+          umma_ts(tmem_O, tmem_P + bj * kPStride + 8 * k, db, C::kIdescPV,
+                  (j > 0 || k > 0) ? 1u : 0u);
         }
         umma_commit(&v_empty[vs]);
         umma_commit(&p_free[bj]);
@@ -353,7 +368,9 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
         const int ks = i % C::kKStages;
         if (!mbar_wait(&k_full[ks], (i / C::kKStages) & 1, s_abort, args.st, 23)) break;
         // S_i overwrites the TMEM buffer that held P_{i-2}: P_{i-2}.V must have completed
-        // (tcgen05 MMAs in flight are not ordered against each other's TMEM accesses)
+        // (tcgen05 MMAs in flight are not ordered against each other's TMEM accesses).  In
+        // decode P has its own buffer, which the softmax rewrites only after S_i is in, so
+        // the same wait orders that rewrite after P_{i-2}.V.
         if (i >= 2 && !mbar_wait(&p_free[b], ((i - 2) >> 1) & 1, s_abort, args.st, 29)) break;
         tc_fence_after();
         const uint32_t sK0 = smem_u32(sK + ks * C::kKVBytes);
@@ -375,179 +392,372 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
   }
   } else {
     regs_raise<C::kRegsSoftmax>();
-    // ---------------- softmax (warps 0 .. 4 kSoftGroups - 1) ----------------
-    // kSoftGroups warpgroups share each row: group sg handles keys [kCols sg, kCols (sg + 1))
-    // of every chunk and dims [kCols sg, ...) of O.  Row maxima are exchanged through shared
-    // memory (double-buffered by chunk parity, one named barrier per chunk); partial row sums
-    // are combined once at the end.  All groups take identical rescale decisions.
-    constexpr int kSG = C::kSoftGroups;
-    constexpr int kCols = 128 / kSG;              // keys (and O dims) per group
-    constexpr int kBlk = kCols / kBlock;          // blocks per group
-    const int wg = warp >> 2;
-    const int quarter = warp & 3;           // TMEM lanes 32q .. 32q+31
-    const int row = quarter * 32 + lane;
-    const int valid_rows = kGroup * ntok;
-    const bool row_ok = row < valid_rows;
-    const bool warp_active = quarter * 32 < valid_rows;
-    const int tr = row_ok ? row / kGroup : 0;
-    const int hr = row % kGroup;
-    const int pos = pos0 + tr;
-    const int tail_u = row_ok ? rec[args.pl.tail_off() + tr] : -1000000;
-    const int tail_last = pos % kBlock;   // keys 0..tail_last of the own block are visible
-    const float sl2 = 1.4426950408889634f * 0.08838834764831845f;   // log2(e)/sqrt(128)
-    float m = -INFINITY, l = 0.f;
-    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t* mrow = masks + tr * mwords;
-    uint32_t mword_next = row_ok ? mrow[c_begin] : 0u;
-    bool ok = true;
-    for (int i = 0; i < nchunks; ++i) {
-      const int b = i & 1;
-      const int q = c_begin + i;
-      const uint32_t mword = (mword_next >> (kBlk * wg)) & ((1u << kBlk) - 1u);   // my blocks
-      if (row_ok && i + 1 < nchunks) mword_next = mrow[q + 1];
-      bool got = ok ? mbar_wait(&s_full[b], (i >> 1) & 1, s_abort, args.st, 24) : false;
-      if (__any_sync(0xffffffffu, !got)) ok = false;   // also reconverges the warp
-      tc_fence_after();
-      uint32_t sv[kCols];
-      const uint32_t ts = tmem + lane_base + b * 128;
-      float mx = -INFINITY;
-      if (ok && warp_active) {
+    if constexpr (kDec) {
+      // ---------------- decode softmax (warps 0 .. 7) ----------------
+      // One query token: its 12 head rows sit in every lane quarter (rows 32q .. 32q+11 hold
+      // copy q), so all eight softmax warps hold valid rows.  Copy q owns keys 16q..16q+15 of
+      // each warpgroup's 64-key half of every chunk and keeps its own running max and sum:
+      // P of a row is zero outside its copy's keys (P lives in its own TMEM columns, zeroed
+      // once; a thread rewrites only its 16 keys), so O row 32q+h accumulates copy q's part
+      // of head h.  The four partial softmaxes are merged by log-sum-exp at the end.  Row
+      // maxima are shared between the two warpgroups as in prefill.
+      static_assert(C::kSoftGroups == 2, "decode softmax assumes two warpgroups");
+      const int wg = warp >> 2;
+      const int quarter = warp & 3;
+      const int row = quarter * 32 + lane;
+      const bool row_ok = lane < kGroup;
+      const int cs = 64 * wg + 16 * quarter;   // my first key column of a chunk
+      const int bs = cs / kBlock;              // my first block slot of a chunk
+      const int tail_u = rec[args.pl.tail_off()];
+      const int tail_last = pos0 % kBlock;
+      const float sl2 = 1.4426950408889634f * 0.08838834764831845f;   // log2(e)/sqrt(128)
+      float m = -INFINITY, l = 0.f;
+      const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+      {
+        uint32_t z[32];
 #pragma unroll
-        for (int c = 0; c < kCols / 32; ++c) tmem_ld32(ts + kCols * wg + 32 * c, sv + 32 * c);
-        tmem_wait_ld();
-        // keys of blocks this row's token did not select -> -inf
-#pragma unroll
-        for (int u = 0; u < kBlk; ++u) {
-          const float bias = ((mword >> u) & 1u) ? 0.f : -INFINITY;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            sv[4 * u + kk] = __float_as_uint(__uint_as_float(sv[4 * u + kk]) + bias);
-        }
-        // the own block: hide the tokens after the query (only where it lies)
-        const int tu = tail_u - q * C::kChunkBlocks - kBlk * wg;
-        if (__any_sync(0xffffffffu, tu >= 0 && tu < kBlk)) {
-#pragma unroll
-          for (int u = 0; u < kBlk; ++u) {
-            if (u == tu) {
-              if (tail_last < 1) sv[4 * u + 1] = __float_as_uint(-INFINITY);
-              if (tail_last < 2) sv[4 * u + 2] = __float_as_uint(-INFINITY);
-              if (tail_last < 3) sv[4 * u + 3] = __float_as_uint(-INFINITY);
-            }
-          }
-        }
-        float mxs[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) mxs[j] = __uint_as_float(sv[j]);
-#pragma unroll
-        for (int j = 8; j < kCols; ++j) mxs[j & 7] = fmaxf(mxs[j & 7], __uint_as_float(sv[j]));
-        mx = fmaxf(fmaxf(fmaxf(mxs[0], mxs[1]), fmaxf(mxs[2], mxs[3])),
-                   fmaxf(fmaxf(mxs[4], mxs[5]), fmaxf(mxs[6], mxs[7])));
-      }
-      // exchange the partial row maxima (every softmax warp takes part, active or not)
-      xmax[(b * kSG + wg) * 128 + row] = mx;
-      tc_fence_before();
-      named_barrier_sync(1, 128 * kSG);
-      tc_fence_after();
-      if (ok && warp_active) {
-#pragma unroll
-        for (int o = 1; o < kSG; ++o) mx = fmaxf(mx, xmax[(b * kSG + ((wg + o) % kSG)) * 128 + row]);
-        const float m_cand = fmaxf(m, mx * sl2);
-        const bool need = m_cand > m + 8.f || (m == -INFINITY && m_cand > -INFINITY);
-        const bool rescale = __any_sync(0xffffffffu, need);
-        float alpha = 1.f;
-        if (rescale) {
-          alpha = (m == -INFINITY) ? 0.f : ex2_approx(m - m_cand);
-          m = m_cand;
-        }
-        const float mneg = (m == -INFINITY) ? 0.f : -m;
-        // P overwrites S in registers: packed pair j lands in sv[j], whose S value (key j) was
-        // consumed at pair j/2 <= j
-        float lsum[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int j = 0; j < kCols / 2; ++j) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * j]), sl2, mneg));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * j + 1]), sl2, mneg));
-          lsum[j & 3] += p0 + p1;
-          sv[j] = pack_bf16x2(p0, p1);
-        }
-        l = l * alpha + ((lsum[0] + lsum[1]) + (lsum[2] + lsum[3]));
-        // packed P of my keys -> columns kCols/2 sg .. of the buffer (every group's S there was
-        // loaded before the barrier above)
-        if constexpr (kCols == 64) {
-          tmem_st32(ts + 32 * wg, sv);
-        } else {
-          tmem_st16(ts + 16 * wg, sv);
-        }
+        for (int j = 0; j < 32; ++j) z[j] = 0u;
+        tmem_st32(tmem_P + lane_base + 32 * wg, z);
+        tmem_st32(tmem_P + lane_base + kPStride + 32 * wg, z);
         tmem_wait_st();
-        if (rescale && i > 0) {
-          // O holds P.V of chunks < i-1 and maybe i-1: wait until chunk i-1 is in, rescale
-          // my dims of O.  P.V of chunk i cannot start before this warp arrives on p_full.
-          const bool gotpv = mbar_wait(pv_done, (i - 1) & 1, s_abort, args.st, 25);
-          if (__any_sync(0xffffffffu, !gotpv)) ok = false;
-          if (ok) {
-            tc_fence_after();
-            const uint32_t to = tmem_O + lane_base + kCols * wg;
+      }
+      uint32_t mword_next = masks[c_begin];
+      bool ok = true;
+      for (int i = 0; i < nchunks; ++i) {
+        const int b = i & 1;
+        const int q = c_begin + i;
+        const uint32_t mword = row_ok ? (mword_next >> bs) & 0xFu : 0u;
+        if (i + 1 < nchunks) mword_next = masks[q + 1];
+        bool got = ok ? mbar_wait(&s_full[b], (i >> 1) & 1, s_abort, args.st, 24) : false;
+        if (__any_sync(0xffffffffu, !got)) ok = false;
+        tc_fence_after();
+        uint32_t sv[16];
+        float mx = -INFINITY;
+        if (ok) {
+          tmem_ld16(tmem + lane_base + b * 128 + cs, sv);
+          tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < kCols / 32; ++c) {
-              uint32_t ov[32];
-              tmem_ld32(to + 32 * c, ov);
-              tmem_wait_ld();
+          for (int u = 0; u < 4; ++u) {
+            const float bias = ((mword >> u) & 1u) ? 0.f : -INFINITY;
 #pragma unroll
-              for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
-              tmem_st32(to + 32 * c, ov);
+            for (int kk = 0; kk < 4; ++kk)
+              sv[4 * u + kk] = __float_as_uint(__uint_as_float(sv[4 * u + kk]) + bias);
+          }
+          // the own block: hide the tokens after the query (only where it lies)
+          const int tu = tail_u - q * C::kChunkBlocks - bs;
+          if (tu >= 0 && tu < 4) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              if (u == tu) {
+                if (tail_last < 1) sv[4 * u + 1] = __float_as_uint(-INFINITY);
+                if (tail_last < 2) sv[4 * u + 2] = __float_as_uint(-INFINITY);
+                if (tail_last < 3) sv[4 * u + 3] = __float_as_uint(-INFINITY);
+              }
             }
-            tmem_wait_st();
+          }
+          float mxs[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) mxs[j] = __uint_as_float(sv[j]);
+#pragma unroll
+          for (int j = 4; j < 16; ++j) mxs[j & 3] = fmaxf(mxs[j & 3], __uint_as_float(sv[j]));
+          mx = fmaxf(fmaxf(mxs[0], mxs[1]), fmaxf(mxs[2], mxs[3]));
+        }
+        xmax[(b * 2 + wg) * 128 + row] = mx;
+        tc_fence_before();
+        named_barrier_sync(1, 256);
+        tc_fence_after();
+        if (ok) {
+          mx = fmaxf(mx, xmax[(b * 2 + (wg ^ 1)) * 128 + row]);
+          const float m_cand = fmaxf(m, mx * sl2);
+          const bool need = m_cand > m + 8.f || (m == -INFINITY && m_cand > -INFINITY);
+          const bool rescale = __any_sync(0xffffffffu, need);
+          float alpha = 1.f;
+          if (rescale) {
+            alpha = (m == -INFINITY) ? 0.f : ex2_approx(m - m_cand);
+            m = m_cand;
+          }
+          const float mneg = (m == -INFINITY) ? 0.f : -m;
+          uint32_t pv[8];
+          float lsum[2] = {0.f, 0.f};
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * j]), sl2, mneg));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * j + 1]), sl2, mneg));
+            lsum[j & 1] += p0 + p1;
+            pv[j] = pack_bf16x2(p0, p1);
+          }
+          l = l * alpha + (lsum[0] + lsum[1]);
+          tmem_st8(tmem_P + lane_base + b * kPStride + cs / 2, pv);
+          tmem_wait_st();
+          if (rescale && i > 0) {
+            // as in prefill: wait until P.V of chunk i-1 is in O, then rescale my dims
+            const bool gotpv = mbar_wait(pv_done, (i - 1) & 1, s_abort, args.st, 25);
+            if (__any_sync(0xffffffffu, !gotpv)) ok = false;
+            if (ok) {
+              tc_fence_after();
+              const uint32_t to = tmem_O + lane_base + 64 * wg;
+#pragma unroll
+              for (int c = 0; c < 2; ++c) {
+                uint32_t ov[32];
+                tmem_ld32(to + 32 * c, ov);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
+                tmem_st32(to + 32 * c, ov);
+              }
+              tmem_wait_st();
+            }
           }
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[b]);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[b]);
-    }
-    // combine the partial row sums
-    xsum[wg * 128 + row] = l;
-    named_barrier_sync(1, 128 * kSG);
-    float l_all = 0.f;
-#pragma unroll
-    for (int o = 0; o < kSG; ++o) l_all += xsum[o * 128 + row];
-    if (ok && nchunks > 0) {
-      // a dedicated barrier: two P.V may still be in flight here, so a parity wait on
-      // pv_done could match an older phase
-      const bool got = mbar_wait(o_final, 0, s_abort, args.st, 26);
+      // merge: each copy's (max, sum, unnormalised O row) goes to shared memory (the K ring is
+      // idle once every P.V has completed), then 192 threads each combine 8 dims of one head
+      xsum[wg * 128 + row] = l;
+      named_barrier_sync(1, 256);
+      const float l_all = xsum[row] + xsum[128 + row];
+      float* mo = reinterpret_cast<float*>(sK);          // [copy][head][128]
+      float* mm = xmax;                                  // [copy][head]: max (log2 domain)
+      float* ml = xmax + 4 * kGroup;                     // [copy][head]: sum
+      const bool got = ok ? mbar_wait(o_final, 0, s_abort, args.st, 26) : false;
       if (!__any_sync(0xffffffffu, !got)) {
         tc_fence_after();
-        if (warp_active) {
-          const uint32_t to = tmem_O + lane_base + kCols * wg;
-          uint32_t ov[kCols];
+        uint32_t ov[64];
+        tmem_ld32(tmem_O + lane_base + 64 * wg, ov);
+        tmem_ld32(tmem_O + lane_base + 64 * wg + 32, ov + 32);
+        tmem_wait_ld();
+        if (row_ok) {
+          const int cr = quarter * kGroup + lane;
+          float4* dst = reinterpret_cast<float4*>(mo + cr * kHeadDim + 64 * wg);
 #pragma unroll
-          for (int c = 0; c < kCols / 32; ++c) tmem_ld32(to + 32 * c, ov + 32 * c);
+          for (int c = 0; c < 16; ++c)
+            dst[c] = make_float4(__uint_as_float(ov[4 * c]), __uint_as_float(ov[4 * c + 1]),
+                                 __uint_as_float(ov[4 * c + 2]), __uint_as_float(ov[4 * c + 3]));
+          if (wg == 0) {
+            mm[cr] = m;
+            ml[cr] = l_all;
+          }
+        }
+      } else {
+        ok = false;
+      }
+      named_barrier_sync(1, 256);
+      const int t = threadIdx.x;
+      if (t < kGroup * 16) {
+        const int h = t / 16, d0 = (t % 16) * 8;
+        float M = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) M = fmaxf(M, mm[c * kGroup + h]);
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        float L = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const float mc = mm[c * kGroup + h];
+          const float f = (mc == -INFINITY) ? 0.f : ex2_approx(mc - M);
+          L += f * ml[c * kGroup + h];
+          const float4* src = reinterpret_cast<const float4*>(mo + (c * kGroup + h) * kHeadDim + d0);
+          const float4 a0 = src[0], a1 = src[1];
+          acc[0] += f * a0.x; acc[1] += f * a0.y; acc[2] += f * a0.z; acc[3] += f * a0.w;
+          acc[4] += f * a1.x; acc[5] += f * a1.y; acc[6] += f * a1.z; acc[7] += f * a1.w;
+        }
+        if (args.splits == 1) {
+          const float inv = L > 0.f ? 1.f / L : 0.f;
+          uint4 v;
+          v.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+          v.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+          v.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
+          v.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+          *reinterpret_cast<uint4*>(args.out + (tok_row0 * kHeads + g * kGroup + h) * kHeadDim +
+                                    d0) = v;
+        } else {
+          const int64_t pr =
+              ((static_cast<int64_t>(tile) * 2 + g) * args.splits + split) * kGroup + h;
+          if (d0 == 0) {
+            args.part_m[pr] = M;
+            args.part_l[pr] = L;
+          }
+          float4* po = reinterpret_cast<float4*>(args.part_o + pr * kHeadDim + d0);
+          po[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+          po[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        }
+      }
+    } else {
+      // ---------------- softmax (warps 0 .. 4 kSoftGroups - 1) ----------------
+      // kSoftGroups warpgroups share each row: group sg handles keys [kCols sg, kCols (sg + 1))
+      // of every chunk and dims [kCols sg, ...) of O.  Row maxima are exchanged through shared
+      // memory (double-buffered by chunk parity, one named barrier per chunk); partial row sums
+      // are combined once at the end.  All groups take identical rescale decisions.
+      constexpr int kSG = C::kSoftGroups;
+      constexpr int kCols = 128 / kSG;              // keys (and O dims) per group
+      constexpr int kBlk = kCols / kBlock;          // blocks per group
+      const int wg = warp >> 2;
+      const int quarter = warp & 3;           // TMEM lanes 32q .. 32q+31
+      const int row = quarter * 32 + lane;
+      const int valid_rows = kGroup * ntok;
+      const bool row_ok = row < valid_rows;
+      const bool warp_active = quarter * 32 < valid_rows;
+      const int tr = row_ok ? row / kGroup : 0;
+      const int hr = row % kGroup;
+      const int pos = pos0 + tr;
+      const int tail_u = row_ok ? rec[args.pl.tail_off() + tr] : -1000000;
+      const int tail_last = pos % kBlock;   // keys 0..tail_last of the own block are visible
+      const float sl2 = 1.4426950408889634f * 0.08838834764831845f;   // log2(e)/sqrt(128)
+      float m = -INFINITY, l = 0.f;
+      const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+      const uint32_t* mrow = masks + tr * mwords;
+      uint32_t mword_next = row_ok ? mrow[c_begin] : 0u;
+      bool ok = true;
+      for (int i = 0; i < nchunks; ++i) {
+        const int b = i & 1;
+        const int q = c_begin + i;
+        const uint32_t mword = (mword_next >> (kBlk * wg)) & ((1u << kBlk) - 1u);   // my blocks
+        if (row_ok && i + 1 < nchunks) mword_next = mrow[q + 1];
+        bool got = ok ? mbar_wait(&s_full[b], (i >> 1) & 1, s_abort, args.st, 24) : false;
+        if (__any_sync(0xffffffffu, !got)) ok = false;   // also reconverges the warp
+        tc_fence_after();
+        uint32_t sv[kCols];
+        const uint32_t ts = tmem + lane_base + b * 128;
+        float mx = -INFINITY;
+        if (ok && warp_active) {
+  #pragma unroll
+          for (int c = 0; c < kCols / 32; ++c) tmem_ld32(ts + kCols * wg + 32 * c, sv + 32 * c);
           tmem_wait_ld();
-          if (row_ok) {
-            if (!args.decode || args.splits == 1) {   // one split: the final output directly
-              const float inv = l_all > 0.f ? 1.f / l_all : 0.f;
-              __nv_bfloat16* o = args.out + ((tok_row0 + tr) * kHeads + g * kGroup + hr) * kHeadDim +
-                                 kCols * wg;
-#pragma unroll
-              for (int c = 0; c < kCols / 8; ++c) {
-                uint4 v;
-                v.x = pack_bf16x2(__uint_as_float(ov[8 * c + 0]) * inv, __uint_as_float(ov[8 * c + 1]) * inv);
-                v.y = pack_bf16x2(__uint_as_float(ov[8 * c + 2]) * inv, __uint_as_float(ov[8 * c + 3]) * inv);
-                v.z = pack_bf16x2(__uint_as_float(ov[8 * c + 4]) * inv, __uint_as_float(ov[8 * c + 5]) * inv);
-                v.w = pack_bf16x2(__uint_as_float(ov[8 * c + 6]) * inv, __uint_as_float(ov[8 * c + 7]) * inv);
-                reinterpret_cast<uint4*>(o)[c] = v;
+          // keys of blocks this row's token did not select -> -inf
+  #pragma unroll
+          for (int u = 0; u < kBlk; ++u) {
+            const float bias = ((mword >> u) & 1u) ? 0.f : -INFINITY;
+  #pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              sv[4 * u + kk] = __float_as_uint(__uint_as_float(sv[4 * u + kk]) + bias);
+          }
+          // the own block: hide the tokens after the query (only where it lies)
+          const int tu = tail_u - q * C::kChunkBlocks - kBlk * wg;
+          if (__any_sync(0xffffffffu, tu >= 0 && tu < kBlk)) {
+  #pragma unroll
+            for (int u = 0; u < kBlk; ++u) {
+              if (u == tu) {
+                if (tail_last < 1) sv[4 * u + 1] = __float_as_uint(-INFINITY);
+                if (tail_last < 2) sv[4 * u + 2] = __float_as_uint(-INFINITY);
+                if (tail_last < 3) sv[4 * u + 3] = __float_as_uint(-INFINITY);
               }
-            } else {
-              const int64_t pr =
-                  ((static_cast<int64_t>(tile) * 2 + g) * args.splits + split) * kGroup + hr;
-              if (wg == 0) {
-                args.part_m[pr] = m;
-                args.part_l[pr] = l_all;
+            }
+          }
+          float mxs[8];
+  #pragma unroll
+          for (int j = 0; j < 8; ++j) mxs[j] = __uint_as_float(sv[j]);
+  #pragma unroll
+          for (int j = 8; j < kCols; ++j) mxs[j & 7] = fmaxf(mxs[j & 7], __uint_as_float(sv[j]));
+          mx = fmaxf(fmaxf(fmaxf(mxs[0], mxs[1]), fmaxf(mxs[2], mxs[3])),
+                     fmaxf(fmaxf(mxs[4], mxs[5]), fmaxf(mxs[6], mxs[7])));
+        }
+        // exchange the partial row maxima (every softmax warp takes part, active or not)
+        xmax[(b * kSG + wg) * 128 + row] = mx;
+        tc_fence_before();
+        named_barrier_sync(1, 128 * kSG);
+        tc_fence_after();
+        if (ok && warp_active) {
+  #pragma unroll
+          for (int o = 1; o < kSG; ++o) mx = fmaxf(mx, xmax[(b * kSG + ((wg + o) % kSG)) * 128 + row]);
+          const float m_cand = fmaxf(m, mx * sl2);
+          const bool need = m_cand > m + 8.f || (m == -INFINITY && m_cand > -INFINITY);
+          const bool rescale = __any_sync(0xffffffffu, need);
+          float alpha = 1.f;
+          if (rescale) {
+            alpha = (m == -INFINITY) ? 0.f : ex2_approx(m - m_cand);
+            m = m_cand;
+          }
+          const float mneg = (m == -INFINITY) ? 0.f : -m;
+          // P overwrites S in registers: packed pair j lands in sv[j], whose S value (key j) was
+          // consumed at pair j/2 <= j
+          float lsum[4] = {0.f, 0.f, 0.f, 0.f};
+  #pragma unroll
+          for (int j = 0; j < kCols / 2; ++j) {
+            const float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * j]), sl2, mneg));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * j + 1]), sl2, mneg));
+            lsum[j & 3] += p0 + p1;
+            sv[j] = pack_bf16x2(p0, p1);
+          }
+          l = l * alpha + ((lsum[0] + lsum[1]) + (lsum[2] + lsum[3]));
+          // packed P of my keys -> columns kCols/2 sg .. of the buffer (every group's S there was
+          // loaded before the barrier above)
+          if constexpr (kCols == 64) {
+            tmem_st32(ts + 32 * wg, sv);
+          } else {
+            tmem_st16(ts + 16 * wg, sv);
+          }
+          tmem_wait_st();
+          if (rescale && i > 0) {
+            // O holds P.V of chunks < i-1 and maybe i-1: wait until chunk i-1 is in, rescale
+            // my dims of O.  P.V of chunk i cannot start before this warp arrives on p_full.
+            const bool gotpv = mbar_wait(pv_done, (i - 1) & 1, s_abort, args.st, 25);
+            if (__any_sync(0xffffffffu, !gotpv)) ok = false;
+            if (ok) {
+              tc_fence_after();
+              const uint32_t to = tmem_O + lane_base + kCols * wg;
+  #pragma unroll
+              for (int c = 0; c < kCols / 32; ++c) {
+                uint32_t ov[32];
+                tmem_ld32(to + 32 * c, ov);
+                tmem_wait_ld();
+  #pragma unroll
+                for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
+                tmem_st32(to + 32 * c, ov);
               }
-              float4* po = reinterpret_cast<float4*>(args.part_o + pr * kHeadDim + kCols * wg);
-#pragma unroll
-              for (int c = 0; c < kCols / 4; ++c)
-                po[c] = make_float4(__uint_as_float(ov[4 * c]), __uint_as_float(ov[4 * c + 1]),
-                                    __uint_as_float(ov[4 * c + 2]), __uint_as_float(ov[4 * c + 3]));
+              tmem_wait_st();
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[b]);
+      }
+      // combine the partial row sums
+      xsum[wg * 128 + row] = l;
+      named_barrier_sync(1, 128 * kSG);
+      float l_all = 0.f;
+  #pragma unroll
+      for (int o = 0; o < kSG; ++o) l_all += xsum[o * 128 + row];
+      if (ok && nchunks > 0) {
+        // a dedicated barrier: two P.V may still be in flight here, so a parity wait on
+        // pv_done could match an older phase
+        const bool got = mbar_wait(o_final, 0, s_abort, args.st, 26);
+        if (!__any_sync(0xffffffffu, !got)) {
+          tc_fence_after();
+          if (warp_active) {
+            const uint32_t to = tmem_O + lane_base + kCols * wg;
+            uint32_t ov[kCols];
+  #pragma unroll
+            for (int c = 0; c < kCols / 32; ++c) tmem_ld32(to + 32 * c, ov + 32 * c);
+            tmem_wait_ld();
+            if (row_ok) {
+              if (!kDec || args.splits == 1) {   // one split: the final output directly
+                const float inv = l_all > 0.f ? 1.f / l_all : 0.f;
+                __nv_bfloat16* o = args.out + ((tok_row0 + tr) * kHeads + g * kGroup + hr) * kHeadDim +
+                                   kCols * wg;
+  #pragma unroll
+                for (int c = 0; c < kCols / 8; ++c) {
+                  uint4 v;
+                  v.x = pack_bf16x2(__uint_as_float(ov[8 * c + 0]) * inv, __uint_as_float(ov[8 * c + 1]) * inv);
+                  v.y = pack_bf16x2(__uint_as_float(ov[8 * c + 2]) * inv, __uint_as_float(ov[8 * c + 3]) * inv);
+                  v.z = pack_bf16x2(__uint_as_float(ov[8 * c + 4]) * inv, __uint_as_float(ov[8 * c + 5]) * inv);
+                  v.w = pack_bf16x2(__uint_as_float(ov[8 * c + 6]) * inv, __uint_as_float(ov[8 * c + 7]) * inv);
+                  reinterpret_cast<uint4*>(o)[c] = v;
+                }
+              } else {
+                const int64_t pr =
+                    ((static_cast<int64_t>(tile) * 2 + g) * args.splits + split) * kGroup + hr;
+                if (wg == 0) {
+                  args.part_m[pr] = m;
+                  args.part_l[pr] = l_all;
+                }
+                float4* po = reinterpret_cast<float4*>(args.part_o + pr * kHeadDim + kCols * wg);
+  #pragma unroll
+                for (int c = 0; c < kCols / 4; ++c)
+                  po[c] = make_float4(__uint_as_float(ov[4 * c]), __uint_as_float(ov[4 * c + 1]),
+                                      __uint_as_float(ov[4 * c + 2]), __uint_as_float(ov[4 * c + 3]));
+              }
             }
           }
         }
