@@ -385,7 +385,7 @@ struct DecodeGeom {
   int64_t ld = 4;
   PlanLayout pl;
   size_t o_scores = 0, o_nc = 0, o_idx = 0, o_cnt = 0, o_plan = 0, o_po = 0, o_pm = 0, o_pl = 0,
-         o_hist = 0, o_ccnt = 0, o_cand = 0, total = 0;
+         o_hist = 0, o_ccnt = 0, o_cand = 0, o_rinfo = 0, total = 0;
   // shared memory of k_topk_finish
   int finish_smem() const {
     return kTopkSharedBytes + cand_cap * 8 + 2 * ((std::max(max_nc, 1) + 31) / 32) * 4;
@@ -424,6 +424,7 @@ qsa_status decode_geom(const qsa_cache* c, const qsa_params& p, DecodeGeom* g) {
   g->o_ccnt = g->o_hist + static_cast<size_t>(g->B) * kTopkBins * 4;
   g->cand_cap = std::min(kCandCap, static_cast<int>(round_up(std::max(g->max_nc, 64), 64)));
   g->o_cand = cv.take(static_cast<size_t>(g->B) * g->cand_cap * 8);
+  g->o_rinfo = cv.take(static_cast<size_t>(g->B) * 4 * 4);   // threshold bin, above, in bin
   g->total = cv.off;
   return QSA_OK;
 }
@@ -687,11 +688,10 @@ qsa_status qsa_append_kv(const qsa_cache* cache, const void* k, const void* v, c
     const int slots = (n_new + 3) / 4 + 1;   // blocks a sequence's new tokens can touch
     const int64_t n = static_cast<int64_t>(p.batch) * n_new * 32 + static_cast<int64_t>(p.batch) * slots * 8;
     const int grid = static_cast<int>(std::min<int64_t>((n + 255) / 256, int64_t(sms) * 16));
-    k_append<<<grid, 256, 0, s>>>(p, slots);
-    QSA_CHECK_LAUNCH();
+    QSA_CHECK_PDL(launch_pdl(k_append, dim3(grid), dim3(256), 0, s, p, slots));
   }
-  k_append_len<<<(p.batch + 255) / 256, 256, 0, s>>>(cache->len, counts, n_new, p.batch);
-  QSA_CHECK_LAUNCH();
+  QSA_CHECK_PDL(launch_pdl(k_append_len, dim3((p.batch + 255) / 256), dim3(256), 0, s, cache->len,
+                           counts, n_new, p.batch));
   return QSA_OK;
 }
 
@@ -729,6 +729,7 @@ qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, 
   uint32_t* hist = reinterpret_cast<uint32_t*>(ws + g.o_hist);
   int32_t* cand_cnt = reinterpret_cast<int32_t*>(ws + g.o_ccnt);
   uint64_t* cand = reinterpret_cast<uint64_t*>(ws + g.o_cand);
+  int32_t* rinfo = reinterpret_cast<int32_t*>(ws + g.o_rinfo);
   const int sms = num_sms();
   const int max_nc_now = (max_len - 1) / 4;
   // the decode kernels form one chain of programmatic dependent launches (each waits for the
@@ -783,12 +784,14 @@ qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, 
   }
   // a3: top-k: candidates at or above the threshold bin, then the exact select per row
   {
-    // one pass of 4096 scores per CTA
-    const int parts = std::max(1, (max_nc_now + 4095) / 4096);
+    // up to one pass of kCollectPerCta scores per CTA, and no more CTAs than one wave (one
+    // CTA per SM: 512 threads of about 120 registers)
+    const int parts = std::max(1, std::min((max_nc_now + kCollectPerCta - 1) / kCollectPerCta,
+                                           sms / g.B));
     QSA_CHECK_PDL(launch_pdl(k_topk_collect, dim3(g.B * parts), dim3(kCandThreads), 0, s,
                              static_cast<const float*>(scores), g.ld,
                              static_cast<const int32_t*>(n_c), g.topk, parts, g.cand_cap,
-                             static_cast<const uint32_t*>(hist), cand_cnt, cand));
+                             static_cast<const uint32_t*>(hist), cand_cnt, cand, rinfo));
     const int smem = g.finish_smem();
     if (!set_smem(k_topk_finish, smem)) return QSA_ERR_CUDA;
     // also writes each sequence's attention plan record
@@ -797,7 +800,8 @@ qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, 
                              static_cast<const int32_t*>(n_c), g.topk, g.cand_cap,
                              std::max(g.max_nc, 1), static_cast<const uint32_t*>(hist),
                              static_cast<const int32_t*>(cand_cnt),
-                             static_cast<const uint64_t*>(cand), idx, cnt,
+                             static_cast<const uint64_t*>(cand),
+                             static_cast<const int32_t*>(rinfo), idx, cnt,
                              static_cast<const int32_t*>(cache->len), g.pl, plan));
   }
   // a6: split attention + combine

@@ -328,6 +328,8 @@ __device__ __forceinline__ void append_kbar_item(const AppendParams& p, int64_t 
 // K/V copies and compressed-key updates in one launch (both read the lengths before the
 // append); k_append_len then advances the lengths.
 __global__ void k_append(AppendParams p, int max_blocks_touched) {
+  pdl_trigger();
+  pdl_wait();   // launched as a programmatic dependent of the caller's last kernel
   const int64_t n_copy = static_cast<int64_t>(p.batch) * p.n_new * 32;
   const int64_t n_kbar = static_cast<int64_t>(p.batch) * max_blocks_touched * 8;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n_copy + n_kbar;
@@ -347,6 +349,8 @@ __global__ void k_zero_words(uint32_t* __restrict__ p, int64_t n) {
 }
 
 __global__ void k_append_len(int32_t* len, const int32_t* counts, int32_t n_new, int batch) {
+  pdl_trigger();
+  pdl_wait();   // every k_append thread has read len
   for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < batch; b += gridDim.x * blockDim.x) {
     int c = counts ? counts[b] : n_new;
     c = c < 0 ? 0 : (c > n_new ? n_new : c);
@@ -555,24 +559,27 @@ __device__ __forceinline__ void topk_row(const float* __restrict__ src, int n, i
 // Long rows (decode): top-k from a first-digit histogram built while scoring, in two steps.
 //   k_topk_collect  (rows x parts CTAs): every CTA finds the threshold bin B1 of its row from
 //                   the histogram and appends (key, index) of each score in bins >= B1 to the
-//                   row's candidate list (at most topk - 1 + hist[B1] entries).
+//                   row's candidate list (at most topk - 1 + hist[B1] entries); the row's first
+//                   CTA also records B1 and the counts above and in it (row info).
 //   k_topk_finish   (one CTA per row): exact radix select among the candidates (digits 2, 3),
 //                   then the ascending index list through shared-memory bitmaps: every key
 //                   above the threshold, plus the lowest-index keys equal to it.
 // A row whose candidates would not fit `cap` is left to the full-row select (topk_row).
-constexpr int kCandThreads = 256;
-static_assert(kCandThreads * 16 == 4096, "hist_threshold_bin gives each thread 16 bins");
+constexpr int kCandThreads = 512;
+constexpr int kCandBins = 4096 / kCandThreads;   // histogram bins per thread
+static_assert(kCandBins % 4 == 0, "hist_threshold_bin loads its bins as uint4");
 
-// Threshold bin of a row from its 4096-bin histogram: thread t holds bins 4080-16t .. 4095-16t
-// in registers (the highest bins go to thread 0).  Returns the bin where the count of keys in
-// higher bins first reaches `topk`; *above receives that count and *in_bin the bin's own.
+// Threshold bin of a row from its 4096-bin histogram: thread t holds bins 4096-kCandBins(t+1)
+// .. 4095-kCandBins t in registers (the highest bins go to thread 0).  Returns the bin where the
+// count of keys in higher bins first reaches `topk`; *above receives that count and *in_bin the
+// bin's own.
 __device__ __forceinline__ int hist_threshold_bin(const uint32_t* __restrict__ h, int topk,
                                                   int* above_out, int* in_bin_out, int* sh /*[40]*/) {
-  const int lo = 4080 - 16 * static_cast<int>(threadIdx.x);
+  const int lo = 4096 - kCandBins * (static_cast<int>(threadIdx.x) + 1);
   const uint4* h4 = reinterpret_cast<const uint4*>(h + lo);
-  uint32_t v[16];
+  uint32_t v[kCandBins];
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
+  for (int q = 0; q < kCandBins / 4; ++q) {
     const uint4 x = h4[q];
     v[4 * q] = x.x;
     v[4 * q + 1] = x.y;
@@ -581,11 +588,11 @@ __device__ __forceinline__ int hist_threshold_bin(const uint32_t* __restrict__ h
   }
   int local = 0;
 #pragma unroll
-  for (int j = 0; j < 16; ++j) local += static_cast<int>(v[j]);
+  for (int j = 0; j < kCandBins; ++j) local += static_cast<int>(v[j]);
   int tot;
   int running = block_excl_scan(local, sh, &tot);   // keys in bins above this thread's range
 #pragma unroll
-  for (int j = 15; j >= 0; --j) {
+  for (int j = kCandBins - 1; j >= 0; --j) {
     const int c = static_cast<int>(v[j]);
     if (running < topk && running + c >= topk) {
       sh[36] = lo + j;
@@ -602,14 +609,17 @@ __device__ __forceinline__ int hist_threshold_bin(const uint32_t* __restrict__ h
   return bin;
 }
 
-// Each CTA covers `per` (a multiple of 4) scores of one row in passes of 16 scores a thread:
+// Each CTA covers `per` (a multiple of 4) scores of one row in passes of 32 scores a thread
+// (one or a few passes):
 // all loads of a pass are issued before one block scan places the pass's candidates, so a
-// pass costs one load latency and one atomic on the row's counter.
-constexpr int kCollectPerThread = 16;
+// pass costs one load latency and one atomic on the row's counter.  Few, large CTAs: a grid
+// of small ones spent most of its time starting them.
+constexpr int kCollectPerThread = 32;
+constexpr int kCollectPerCta = kCandThreads * kCollectPerThread;   // one pass
 __global__ void __launch_bounds__(kCandThreads) k_topk_collect(
     const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_c, int topk,
     int parts, int cap, const uint32_t* __restrict__ hist, int32_t* __restrict__ cand_cnt,
-    uint64_t* __restrict__ cand) {
+    uint64_t* __restrict__ cand, int32_t* __restrict__ rinfo) {
   pdl_trigger();
   pdl_wait();
   __shared__ int sh[40];
@@ -620,6 +630,11 @@ __global__ void __launch_bounds__(kCandThreads) k_topk_collect(
   int above, in_b1;
   const uint32_t b1 = static_cast<uint32_t>(
       hist_threshold_bin(hist + static_cast<int64_t>(r) * 4096, topk, &above, &in_b1, sh));
+  if (part == 0 && threadIdx.x == 0) {
+    rinfo[4 * r] = static_cast<int32_t>(b1);
+    rinfo[4 * r + 1] = above;
+    rinfo[4 * r + 2] = in_b1;
+  }
   if (above + in_b1 > cap) return;   // overflow: the finish kernel takes the full-row path
   const int per = ((n + parts - 1) / parts + 3) & ~3;
   const int a = part * per, e = min(n, a + per);
@@ -750,8 +765,9 @@ __device__ __forceinline__ void topk_select_candidates(TopkShared& S, const uint
 __global__ void __launch_bounds__(kTopkThreads) k_topk_finish(
     const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_c, int topk,
     int cap, int n_max, const uint32_t* __restrict__ hist, const int32_t* __restrict__ cand_cnt,
-    const uint64_t* __restrict__ cand, int32_t* __restrict__ idx, int32_t* __restrict__ cnt,
-    const int32_t* __restrict__ len, PlanLayout pl, int32_t* __restrict__ plan) {
+    const uint64_t* __restrict__ cand, const int32_t* __restrict__ rinfo,
+    int32_t* __restrict__ idx, int32_t* __restrict__ cnt, const int32_t* __restrict__ len,
+    PlanLayout pl, int32_t* __restrict__ plan) {
   pdl_trigger();
   pdl_wait();
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -774,13 +790,11 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk_finish(
     return;
   }
   const uint32_t* h = hist + static_cast<int64_t>(r) * 4096;
-  for (int i = tid; i < kTopkBins; i += blockDim.x) S.hist[i] = h[i];
-  __syncthreads();
-  int above;
-  const uint32_t b1 = static_cast<uint32_t>(topk_find_bin(S, kTopkBins, topk, &above));
+  // the threshold bin and its counts, as the collect kernel found them in the histogram
+  const uint32_t b1 = static_cast<uint32_t>(rinfo[4 * r]);
+  const int above = rinfo[4 * r + 1];
+  const int in_b1 = rinfo[4 * r + 2];
   const int C = cand_cnt[r];
-  const int in_b1 = static_cast<int>(S.hist[b1]);
-  __syncthreads();   // every thread has read the histogram before it is rewritten
   if (above + in_b1 > cap || C > cap) {
     // the candidates did not fit: full-row radix select on the scores in global memory
     topk_row(scores + static_cast<int64_t>(r) * ld, n, topk, h, out, S);
