@@ -785,7 +785,7 @@ qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, 
   // a3: top-k: candidates at or above the threshold bin, then the exact select per row
   {
     // up to one pass of kCollectPerCta scores per CTA, and no more CTAs than one wave (one
-    // CTA per SM: 512 threads of about 120 registers)
+    // CTA of 512 threads per SM)
     const int parts = std::max(1, std::min((max_nc_now + kCollectPerCta - 1) / kCollectPerCta,
                                            sms / g.B));
     QSA_CHECK_PDL(launch_pdl(k_topk_collect, dim3(g.B * parts), dim3(kCandThreads), 0, s,

@@ -609,14 +609,14 @@ __device__ __forceinline__ int hist_threshold_bin(const uint32_t* __restrict__ h
   return bin;
 }
 
-// Each CTA covers `per` (a multiple of 4) scores of one row in passes of 32 scores a thread
-// (one or a few passes):
-// all loads of a pass are issued before one block scan places the pass's candidates, so a
-// pass costs one load latency and one atomic on the row's counter.  Few, large CTAs: a grid
-// of small ones spent most of its time starting them.
-constexpr int kCollectPerThread = 32;
+// Each CTA covers `per` (a multiple of 4) scores of one row in passes of 64 scores a thread
+// (usually one pass).  The first pass's loads go out before the threshold bin is looked up in
+// the histogram, so that lookup hides under them; after the loads one block scan places the
+// pass's candidates with a single atomic on the row's counter.  Few, large CTAs: a grid of
+// small ones spent most of its time starting them.
+constexpr int kCollectPerThread = 64;
 constexpr int kCollectPerCta = kCandThreads * kCollectPerThread;   // one pass
-__global__ void __launch_bounds__(kCandThreads) k_topk_collect(
+__global__ void __launch_bounds__(kCandThreads, 1) k_topk_collect(
     const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_c, int topk,
     int parts, int cap, const uint32_t* __restrict__ hist, int32_t* __restrict__ cand_cnt,
     uint64_t* __restrict__ cand, int32_t* __restrict__ rinfo) {
@@ -627,21 +627,12 @@ __global__ void __launch_bounds__(kCandThreads) k_topk_collect(
   const int r = blockIdx.x / parts, part = blockIdx.x % parts;
   const int n = n_c[r];
   if (n <= topk) return;
-  int above, in_b1;
-  const uint32_t b1 = static_cast<uint32_t>(
-      hist_threshold_bin(hist + static_cast<int64_t>(r) * 4096, topk, &above, &in_b1, sh));
-  if (part == 0 && threadIdx.x == 0) {
-    rinfo[4 * r] = static_cast<int32_t>(b1);
-    rinfo[4 * r + 1] = above;
-    rinfo[4 * r + 2] = in_b1;
-  }
-  if (above + in_b1 > cap) return;   // overflow: the finish kernel takes the full-row path
   const int per = ((n + parts - 1) / parts + 3) & ~3;
   const int a = part * per, e = min(n, a + per);
   const float* src = scores + static_cast<int64_t>(r) * ld;
   uint64_t* out = cand + static_cast<int64_t>(r) * cap;
-  constexpr int kPass = kCandThreads * kCollectPerThread;
-  for (int base = a; base < e; base += kPass) {
+  uint32_t b1 = 0;
+  for (int base = a; base < e; base += kCollectPerCta) {
     float x[kCollectPerThread];
 #pragma unroll
     for (int q = 0; q < kCollectPerThread / 4; ++q) {
@@ -653,21 +644,32 @@ __global__ void __launch_bounds__(kCandThreads) k_topk_collect(
       x[4 * q + 2] = f.z;
       x[4 * q + 3] = f.w;
     }
-    uint32_t take = 0;
+    if (base == a) {
+      int above, in_b1;
+      b1 = static_cast<uint32_t>(
+          hist_threshold_bin(hist + static_cast<int64_t>(r) * 4096, topk, &above, &in_b1, sh));
+      if (part == 0 && threadIdx.x == 0) {
+        rinfo[4 * r] = static_cast<int32_t>(b1);
+        rinfo[4 * r + 1] = above;
+        rinfo[4 * r + 2] = in_b1;
+      }
+      if (above + in_b1 > cap) return;   // overflow: the finish kernel takes the full-row path
+    }
+    uint64_t take = 0;
 #pragma unroll
     for (int j = 0; j < kCollectPerThread; ++j) {
       const int i = base + 4 * ((j / 4) * kCandThreads + static_cast<int>(threadIdx.x)) + (j & 3);
-      if (i < e && (float_key(x[j]) >> 20) >= b1) take |= 1u << j;
+      if (i < e && (float_key(x[j]) >> 20) >= b1) take |= 1ull << j;
     }
     int tot;
-    const int ex = block_excl_scan(__popc(take), sh, &tot);
+    const int ex = block_excl_scan(__popcll(take), sh, &tot);
     if (tot == 0) continue;   // uniform: tot is the block total
     if (threadIdx.x == 0) s_base = atomicAdd(cand_cnt + r, tot);
     __syncthreads();
     int slot = s_base + ex;
 #pragma unroll
     for (int j = 0; j < kCollectPerThread; ++j) {
-      if (take & (1u << j)) {
+      if (take & (1ull << j)) {
         const int i = base + 4 * ((j / 4) * kCandThreads + static_cast<int>(threadIdx.x)) + (j & 3);
         if (slot < cap) out[slot] = (static_cast<uint64_t>(float_key(x[j])) << 32) | static_cast<uint32_t>(i);
         ++slot;
