@@ -202,7 +202,16 @@ def run_qsa(args, rank, world, local):
         if args.decode_batch != spec.batch:   # smaller case of the same workload (captures)
             spec.batch = args.decode_batch
             spec.context = [262140 + (i % 4) for i in range(spec.batch)]
-        cache = qsa.KVCache(spec.batch, spec.capacity, dev, zero=False)
+        if args.paged_tokens:
+            # paged cache: every sequence's pages are drawn from a seeded shuffle of the pool
+            max_pages = spec.capacity // args.paged_tokens
+            pool = spec.batch * max_pages
+            perm = torch.randperm(pool, generator=torch.Generator().manual_seed(4242 + rank))
+            table = perm.view(spec.batch, max_pages).to(torch.int32).to(dev)
+            cache = qsa.PagedKVCache(spec.batch, spec.capacity, args.paged_tokens, pool, table,
+                                     dev, zero=False)
+        else:
+            cache = qsa.KVCache(spec.batch, spec.capacity, dev, zero=False)
         kc, vc, kic = W.decode_context(spec, device=dev)
         lmax = max(spec.context)
         for c0 in range(0, lmax, 16384):
@@ -410,6 +419,9 @@ def main():
     ap.add_argument("--rows-per-tile", type=int, default=0)
     ap.add_argument("--chunk-rows", type=int, default=0)
     ap.add_argument("--decode-splits", type=int, default=0)
+    ap.add_argument("--paged-tokens", type=int, default=0,
+                    help="decode from a paged cache with pages of this many tokens (a multiple "
+                         "of 512); 0 = contiguous cache")
     ap.add_argument("--decode-batch", type=int, default=DEC_BATCH,
                     help="sequences of the 256K-context decode batch (64 = the workload)")
     ap.add_argument("--prefill-len", type=int, default=PREFILL_T,
@@ -478,7 +490,9 @@ def main():
                  "dtype": "bf16", "data": "synthetic",
                  "config": {"workload": " + ".join(
                                 ([f"qsa_prefill_{args.prefill_len // 1024}k"] if r["do_prefill"] else [])
-                                + ([f"qsa_decode_256k_b{args.decode_batch}"] if r["do_decode"] else [])),
+                                + ([f"qsa_decode_256k_b{args.decode_batch}"
+                                    + (f"_paged{args.paged_tokens}" if args.paged_tokens else "")]
+                                   if r["do_decode"] else [])),
                             "prefill_seq_len": args.prefill_len, "decode_batch": args.decode_batch,
                             "decode_context": "262140 + (i mod 4)", "topk_blocks": TOPK,
                             "heads": "24q/2kv", "head_dim": 128, "indexer": "16x64",

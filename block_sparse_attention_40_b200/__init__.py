@@ -4,5 +4,5 @@ The kernels and the C ABI live in ``csrc/`` and build into ``lib/libqsa.so`` (de
 ``include/qsa.h``).  ``binding`` is the thin ctypes layer that tests and benchmarks call;
 ``workloads`` draws the seeded synthetic inputs.
 """
-from .binding import (KVCache, Decoder, Prefill, QSAError, compress, index_scores,  # noqa: F401
+from .binding import (KVCache, PagedKVCache, Decoder, Prefill, QSAError, compress, index_scores,  # noqa: F401
                       last_device_error, load, prefill, prefill_select, topk, version)

@@ -30,7 +30,8 @@ EXPORTS = ("qsa_status_string", "qsa_version", "qsa_launch_count", "qsa_workspac
            "qsa_compress_workspace_size", "qsa_compress", "qsa_index_scores", "qsa_topk",
            "qsa_prefill_workspace_size", "qsa_prefill", "qsa_prefill_select",
            "qsa_sparse_attention", "qsa_append_kv", "qsa_decode_workspace_size", "qsa_decode",
-           "qsa_decode_noalloc")
+           "qsa_decode_noalloc", "qsa_append_kv_paged", "qsa_decode_paged_workspace_size",
+           "qsa_decode_paged")
 
 
 class QSAError(RuntimeError):
@@ -48,6 +49,11 @@ class CacheDesc(ctypes.Structure):
     _fields_ = [("k_blocks", ctypes.c_void_p), ("v_blocks", ctypes.c_void_p),
                 ("kbar", ctypes.c_void_p), ("kbar_partial", ctypes.c_void_p),
                 ("len", ctypes.c_void_p), ("batch", ctypes.c_int32), ("capacity", ctypes.c_int32)]
+
+
+class PagedCacheDesc(ctypes.Structure):
+    _fields_ = [("base", CacheDesc), ("page_table", ctypes.c_void_p),
+                ("page_tokens", ctypes.c_int32), ("pool_pages", ctypes.c_int32)]
 
 
 _lock = threading.Lock()
@@ -86,6 +92,9 @@ def load(build_if_needed: bool = True):
             "qsa_decode_workspace_size": ([P, Params], SZ),
             "qsa_decode": ([P, P, P, P, P, P, P, P, P, SZ, Params, P], st),
             "qsa_decode_noalloc": ([P, P, P, P, P, P, P, P, Params, P], st),
+            "qsa_append_kv_paged": ([P, P, P, P, I32, P, P, P], st),
+            "qsa_decode_paged_workspace_size": ([P, Params], SZ),
+            "qsa_decode_paged": ([P, P, P, P, P, P, P, P, P, SZ, Params, P], st),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -323,6 +332,10 @@ def prefill_select(q_idx, k_idx, w, cu_seqlens, topk=512):
 class KVCache:
     """Caller-owned decode cache (torch-allocated buffers, blocked layout of include/qsa.h)."""
 
+    _append_fn = "qsa_append_kv"
+    _ws_fn = "qsa_decode_workspace_size"
+    _decode_fn = "qsa_decode"
+
     def __init__(self, batch: int, capacity: int, device, zero=True):
         if capacity % BLOCK:
             raise ValueError("capacity must be a multiple of 4")
@@ -343,6 +356,15 @@ class KVCache:
                          self.kbar_partial.data_ptr(), self.len.data_ptr(), self.batch,
                          self.capacity)
 
+    def kbar_rows(self, b: int, n: int) -> torch.Tensor:
+        """Compressed keys of blocks 0 .. n-1 of sequence b, [n, 64] (a view or a gather)."""
+        return self.kbar[b, :n]
+
+    def kv_rows(self, b: int, g: int, n: int):
+        """K and V rows of tokens 0 .. n-1 of sequence b, KV head g: two [n, 128] tensors."""
+        return (self.k_blocks[b, g].reshape(-1, HEAD_DIM)[:n],
+                self.v_blocks[b, g].reshape(-1, HEAD_DIM)[:n])
+
     def append(self, k, v, k_idx, counts: Optional[Sequence[int]] = None):
         """Append k, v [B, n, 2, 128] and k_idx [B, n, 64] (counts[b] <= n tokens each)."""
         _need(k, "k", torch.bfloat16, (NUM_KV_HEADS, HEAD_DIM), 4)
@@ -357,7 +379,8 @@ class KVCache:
             d_counts = torch.tensor(counts, dtype=torch.int32, device=self.device)
         h_len = (ctypes.c_int32 * self.batch)(*self.h_len)
         desc = self.desc()
-        _check("qsa_append_kv", load().qsa_append_kv(
+        name = self._append_fn
+        _check(name, getattr(load(), name)(
             ctypes.byref(desc), _ptr(k), _ptr(v), _ptr(k_idx), int(n), _ptr(d_counts), h_len,
             _stream(self.device)))
         for b in range(self.batch):
@@ -366,8 +389,57 @@ class KVCache:
         return self
 
 
+class PagedKVCache(KVCache):
+    """Caller-owned paged decode cache: sequence b's logical page j (tokens j*page_tokens ..)
+    lives in pool page page_table[b, j] (layout of qsa_paged_cache in include/qsa.h)."""
+
+    _append_fn = "qsa_append_kv_paged"
+    _ws_fn = "qsa_decode_paged_workspace_size"
+    _decode_fn = "qsa_decode_paged"
+
+    def __init__(self, batch: int, capacity: int, page_tokens: int, pool_pages: int,
+                 page_table: torch.Tensor, device, zero=True):
+        if page_tokens % 512 or capacity % page_tokens:
+            raise ValueError("page_tokens must be a multiple of 512 dividing the capacity")
+        if (page_table.dtype != torch.int32 or page_table.device != torch.device(device)
+                or tuple(page_table.shape) != (batch, capacity // page_tokens)):
+            raise ValueError("page_table must be int32 [batch, capacity // page_tokens] on the "
+                             "cache's device")
+        alloc = torch.zeros if zero else torch.empty
+        self.batch, self.capacity, self.device = int(batch), int(capacity), torch.device(device)
+        self.page_tokens, self.pool_pages = int(page_tokens), int(pool_pages)
+        self.page_table = page_table.contiguous()
+        nb = page_tokens // BLOCK
+        self.k_blocks = alloc((pool_pages, NUM_KV_HEADS, nb, BLOCK, HEAD_DIM),
+                              dtype=torch.bfloat16, device=device)
+        self.v_blocks = alloc((pool_pages, NUM_KV_HEADS, nb, BLOCK, HEAD_DIM),
+                              dtype=torch.bfloat16, device=device)
+        self.kbar = alloc((pool_pages, nb, IDX_DIM), dtype=torch.bfloat16, device=device)
+        self.kbar_partial = torch.zeros((batch, IDX_DIM), dtype=torch.float32, device=device)
+        self.len = torch.zeros((batch,), dtype=torch.int32, device=device)
+        self.h_len = [0] * batch
+
+    def desc(self) -> PagedCacheDesc:
+        base = CacheDesc(self.k_blocks.data_ptr(), self.v_blocks.data_ptr(), self.kbar.data_ptr(),
+                         self.kbar_partial.data_ptr(), self.len.data_ptr(), self.batch,
+                         self.capacity)
+        return PagedCacheDesc(base, self.page_table.data_ptr(), self.page_tokens,
+                              self.pool_pages)
+
+    def _pages(self, b: int, n_tokens: int):
+        return self.page_table[b, :(n_tokens + self.page_tokens - 1) // self.page_tokens].long()
+
+    def kbar_rows(self, b: int, n: int) -> torch.Tensor:
+        return self.kbar[self._pages(b, 4 * n)].reshape(-1, IDX_DIM)[:n]
+
+    def kv_rows(self, b: int, g: int, n: int):
+        pages = self._pages(b, n)
+        return (self.k_blocks[pages, g].reshape(-1, HEAD_DIM)[:n],
+                self.v_blocks[pages, g].reshape(-1, HEAD_DIM)[:n])
+
+
 class Decoder:
-    """Reusable decode context for one cache: holds the workspace."""
+    """Reusable decode context for one cache (contiguous or paged): holds the workspace."""
 
     def __init__(self, cache: KVCache, topk=512, decode_splits=0):
         self.cache = cache
@@ -375,9 +447,9 @@ class Decoder:
         self.topk = int(topk)
         self.lib = load()
         desc = cache.desc()
-        n = self.lib.qsa_decode_workspace_size(ctypes.byref(desc), self.params)
+        n = getattr(self.lib, cache._ws_fn)(ctypes.byref(desc), self.params)
         if n == 0:
-            raise QSAError("qsa_decode_workspace_size", 1)
+            raise QSAError(cache._ws_fn, 1)
         self.ws = new_workspace(n, cache.device)
 
     def run(self, q, q_idx, w, out=None, with_selection=False):
@@ -395,7 +467,8 @@ class Decoder:
             cnt = torch.empty((B,), dtype=torch.int32, device=q.device)
         h_len = (ctypes.c_int32 * B)(*self.cache.h_len)
         desc = self.cache.desc()
-        _check("qsa_decode", self.lib.qsa_decode(
+        name = self.cache._decode_fn
+        _check(name, getattr(self.lib, name)(
             _ptr(q), ctypes.byref(desc), _ptr(q_idx), _ptr(w), _ptr(out), h_len, _ptr(idx),
             _ptr(cnt), _ptr(self.ws), self.ws.numel(), self.params, _stream(q.device)))
         return (out, idx, cnt) if with_selection else out
@@ -407,6 +480,8 @@ class Decoder:
 def decode_noalloc(cache: KVCache, q, q_idx, w, topk=512, decode_splits=0, out=None):
     """Decode through qsa_decode_noalloc: no workspace is passed; the library uses its own
     fixed device scratch.  Calls must not overlap on the GPU (they share that scratch)."""
+    if isinstance(cache, PagedKVCache):
+        raise TypeError("qsa_decode_noalloc takes a contiguous cache")
     B = cache.batch
     _need(q, "q", torch.bfloat16, (NUM_HEADS, HEAD_DIM), 3)
     _need(q_idx, "q_idx", torch.bfloat16, (IDX_HEADS, IDX_DIM), 3)

@@ -304,7 +304,8 @@ qsa_status prepare_attention() {
   if (r == 0) {
     r = 1;
     for (const void* fn : {reinterpret_cast<const void*>(k_sparse_attn<false>),
-                           reinterpret_cast<const void*>(k_sparse_attn<true>)}) {
+                           reinterpret_cast<const void*>(k_sparse_attn<true>),
+                           reinterpret_cast<const void*>(k_sparse_attn<true, true>)}) {
       cudaFuncAttributes fa{};
       if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) return QSA_ERR_CUDA;
       if (static_cast<int64_t>(fa.numRegs) * AttnCfg::kThreads < AttnCfg::kRegsNeeded) {
@@ -318,6 +319,7 @@ qsa_status prepare_attention() {
   if (r != 1) return QSA_ERR_UNSUPPORTED;
   if (!set_smem(k_sparse_attn<false>, AttnCfg::kSmemBytes)) return QSA_ERR_CUDA;
   if (!set_smem(k_sparse_attn<true>, AttnCfg::kSmemBytes)) return QSA_ERR_CUDA;
+  if (!set_smem(k_sparse_attn<true, true>, AttnCfg::kSmemBytes)) return QSA_ERR_CUDA;
   return QSA_OK;
 }
 
@@ -375,6 +377,44 @@ qsa_status check_prefill_ptrs(std::initializer_list<const void*> ptrs) {
     if (!p) return QSA_ERR_INVALID_ARG;
     if (!aligned16(p)) return QSA_ERR_ALIGNMENT;
   }
+  return QSA_OK;
+}
+
+// ---- decode caches: contiguous or paged ---------------------------------------------------
+// Both kinds are handled by one implementation through Paging (qsa_common.cuh): a contiguous
+// cache is a pool of one page per sequence, holding its whole capacity.
+struct CacheView {
+  const qsa_cache* c = nullptr;   // pointers, batch, logical capacity
+  Paging pg{};
+  int64_t kv_rows = 0;            // rows of 128 dims in the K (and the V) pool
+  int64_t kbar_rows = 0;          // rows of 64 dims in the compressed-key pool
+};
+
+CacheView contiguous_view(const qsa_cache* c) {
+  CacheView v;
+  v.c = c;
+  v.pg = Paging{nullptr, 1, c->capacity / kBlock, c->batch};
+  v.kv_rows = static_cast<int64_t>(c->batch) * 2 * c->capacity;
+  v.kbar_rows = static_cast<int64_t>(c->batch) * (c->capacity / kBlock);
+  return v;
+}
+
+// The base fields are checked where they are used (append, decode geometry); this checks the
+// paging fields.
+qsa_status paged_view(const qsa_paged_cache* pc, CacheView* v) {
+  if (!pc || !pc->page_table) return QSA_ERR_INVALID_ARG;
+  const qsa_cache* c = &pc->base;
+  if (pc->page_tokens <= 0 || pc->page_tokens % 512 != 0 || pc->pool_pages <= 0 ||
+      c->capacity <= 0 || c->capacity % pc->page_tokens != 0)
+    return QSA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(pc->page_table) % 4 != 0) return QSA_ERR_ALIGNMENT;
+  const int64_t kv_rows = static_cast<int64_t>(pc->pool_pages) * 2 * pc->page_tokens;
+  if (kv_rows >= 0x7fffffffll) return QSA_ERR_UNSUPPORTED;   // TMA row coordinates are int32
+  v->c = c;
+  v->pg = Paging{pc->page_table, c->capacity / pc->page_tokens, pc->page_tokens / kBlock,
+                 pc->pool_pages};
+  v->kv_rows = kv_rows;
+  v->kbar_rows = static_cast<int64_t>(pc->pool_pages) * (pc->page_tokens / kBlock);
   return QSA_OK;
 }
 
@@ -652,9 +692,13 @@ qsa_status qsa_sparse_attention(const void* q, const void* k, const void* v, con
 }
 
 // ---- append ------------------------------------------------------------------------------
-qsa_status qsa_append_kv(const qsa_cache* cache, const void* k, const void* v, const void* k_idx,
-                         int32_t n_new, const int32_t* counts, const int32_t* h_len,
-                         qsa_stream_t stream) {
+}  // extern "C"
+
+namespace {
+qsa_status append_impl(const CacheView& view, const void* k, const void* v, const void* k_idx,
+                       int32_t n_new, const int32_t* counts, const int32_t* h_len,
+                       qsa_stream_t stream) {
+  const qsa_cache* cache = view.c;
   if (!cache || !h_len) return QSA_ERR_INVALID_ARG;
   qsa_status st = check_prefill_ptrs({k, v, k_idx, cache->k_blocks, cache->v_blocks, cache->kbar,
                                       cache->kbar_partial, cache->len});
@@ -682,6 +726,7 @@ qsa_status qsa_append_kv(const qsa_cache* cache, const void* k, const void* v, c
   p.kbar = reinterpret_cast<uint4*>(cache->kbar);
   p.partial = cache->kbar_partial;
   p.len = cache->len;
+  p.pg = view.pg;
   p.st = DevStatus{nullptr};
   const int sms = num_sms();
   {
@@ -694,6 +739,25 @@ qsa_status qsa_append_kv(const qsa_cache* cache, const void* k, const void* v, c
                            counts, n_new, p.batch));
   return QSA_OK;
 }
+}  // namespace
+
+extern "C" {
+
+qsa_status qsa_append_kv(const qsa_cache* cache, const void* k, const void* v, const void* k_idx,
+                         int32_t n_new, const int32_t* counts, const int32_t* h_len,
+                         qsa_stream_t stream) {
+  if (!cache) return QSA_ERR_INVALID_ARG;
+  return append_impl(contiguous_view(cache), k, v, k_idx, n_new, counts, h_len, stream);
+}
+
+qsa_status qsa_append_kv_paged(const qsa_paged_cache* cache, const void* k, const void* v,
+                               const void* k_idx, int32_t n_new, const int32_t* counts,
+                               const int32_t* h_len, qsa_stream_t stream) {
+  CacheView view;
+  const qsa_status st = paged_view(cache, &view);
+  if (st != QSA_OK) return st;
+  return append_impl(view, k, v, k_idx, n_new, counts, h_len, stream);
+}
 
 // ---- decode --------------------------------------------------------------------------------
 size_t qsa_decode_workspace_size(const qsa_cache* cache, qsa_params params) {
@@ -702,9 +766,18 @@ size_t qsa_decode_workspace_size(const qsa_cache* cache, qsa_params params) {
   return g.total;
 }
 
-qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, const void* w,
-                      void* out, const int32_t* h_len, int32_t* sel_idx, int32_t* sel_cnt,
-                      void* workspace, size_t ws_bytes, qsa_params params, qsa_stream_t stream) {
+size_t qsa_decode_paged_workspace_size(const qsa_paged_cache* cache, qsa_params params) {
+  CacheView view;
+  if (paged_view(cache, &view) != QSA_OK) return 0;
+  return qsa_decode_workspace_size(&cache->base, params);
+}
+}  // extern "C"
+
+namespace {
+qsa_status decode_impl(const void* q, const CacheView& view, const void* q_idx, const void* w,
+                       void* out, const int32_t* h_len, int32_t* sel_idx, int32_t* sel_cnt,
+                       void* workspace, size_t ws_bytes, qsa_params params, qsa_stream_t stream) {
+  const qsa_cache* cache = view.c;
   if (!cache || !h_len) return QSA_ERR_INVALID_ARG;
   qsa_status st = check_prefill_ptrs({q, q_idx, w, out, workspace, cache->k_blocks,
                                       cache->v_blocks, cache->kbar, cache->len});
@@ -742,7 +815,7 @@ qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, 
   // a2: scores, with the first radix digit's histogram of every row (one token x 16 heads per sequence, split over M-tiles)
   {
     CUtensorMap tm_kbar, tm_qidx;
-    const uint64_t dk[2] = {64, static_cast<uint64_t>(g.B) * (g.cap / 4)};
+    const uint64_t dk[2] = {64, static_cast<uint64_t>(view.kbar_rows)};
     const uint64_t sk[1] = {128};
     const uint32_t bk[2] = {64, 128};
     if (!make_tmap(&tm_kbar, cache->kbar, 2, dk, sk, bk)) return QSA_ERR_CUDA;
@@ -773,6 +846,8 @@ qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, 
     a.splits = splits;
     a.mtiles_per_split = per;
     a.kbar_rows_per_seq = g.cap / 4;
+    a.pg = view.pg;
+    a.kbar_oob_row = static_cast<int32_t>(view.kbar_rows);
     a.n_c_out = n_c;
     a.hist = hist;
     a.w = reinterpret_cast<const __nv_bfloat16*>(w);
@@ -811,7 +886,7 @@ qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, 
     const uint64_t sq[2] = {256, 24 * 256};
     const uint32_t bq[3] = {64, 12, 1};
     if (!make_tmap(&maps.q, q, 3, dq, sq, bq)) return QSA_ERR_CUDA;
-    const uint64_t dkv[2] = {128, static_cast<uint64_t>(g.B) * 2 * g.cap};
+    const uint64_t dkv[2] = {128, static_cast<uint64_t>(view.kv_rows)};
     const uint64_t skv[1] = {256};
     for (int j = 0; j < kNumBoxSizes; ++j) {
       const uint32_t bkv[2] = {64, 4u << j};
@@ -823,8 +898,9 @@ qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, 
     if (pst != QSA_OK) return pst;
   }
     AttnArgs a{};
-    if (static_cast<uint64_t>(g.B) * 2 * g.cap >= 0x7fffffffull) return QSA_ERR_UNSUPPORTED;
-    a.oob_row = static_cast<int32_t>(static_cast<int64_t>(g.B) * 2 * g.cap);
+    if (view.kv_rows >= 0x7fffffffll) return QSA_ERR_UNSUPPORTED;
+    a.oob_row = static_cast<int32_t>(view.kv_rows);
+    a.pg = view.pg;
     a.plan = plan;
     a.pl = g.pl;
     a.decode = 1;
@@ -836,8 +912,13 @@ qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, 
     a.st = dev_status(ws);
     dim3 grid(g.B, 2, g.splits);
     a.out = reinterpret_cast<__nv_bfloat16*>(out);   // written directly with one split
-    QSA_CHECK_PDL(launch_pdl(k_sparse_attn<true>, grid, dim3(AttnCfg::kThreads), AttnCfg::kSmemBytes,
-                             s, maps, a));
+    if (view.pg.table != nullptr) {
+      QSA_CHECK_PDL(launch_pdl(k_sparse_attn<true, true>, grid, dim3(AttnCfg::kThreads),
+                               AttnCfg::kSmemBytes, s, maps, a));
+    } else {
+      QSA_CHECK_PDL(launch_pdl(k_sparse_attn<true>, grid, dim3(AttnCfg::kThreads),
+                               AttnCfg::kSmemBytes, s, maps, a));
+    }
     if (g.splits > 1) {
       const int warps = g.B * kHeads;
       QSA_CHECK_PDL(launch_pdl(k_decode_combine, dim3((warps * 32 + 255) / 256), dim3(256), 0, s,
@@ -848,6 +929,28 @@ qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, 
     }
   }
   return QSA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+qsa_status qsa_decode(const void* q, const qsa_cache* cache, const void* q_idx, const void* w,
+                      void* out, const int32_t* h_len, int32_t* sel_idx, int32_t* sel_cnt,
+                      void* workspace, size_t ws_bytes, qsa_params params, qsa_stream_t stream) {
+  if (!cache) return QSA_ERR_INVALID_ARG;
+  return decode_impl(q, contiguous_view(cache), q_idx, w, out, h_len, sel_idx, sel_cnt, workspace,
+                     ws_bytes, params, stream);
+}
+
+qsa_status qsa_decode_paged(const void* q, const qsa_paged_cache* cache, const void* q_idx,
+                            const void* w, void* out, const int32_t* h_len, int32_t* sel_idx,
+                            int32_t* sel_cnt, void* workspace, size_t ws_bytes, qsa_params params,
+                            qsa_stream_t stream) {
+  CacheView view;
+  const qsa_status st = paged_view(cache, &view);
+  if (st != QSA_OK) return st;
+  return decode_impl(q, view, q_idx, w, out, h_len, sel_idx, sel_cnt, workspace, ws_bytes, params,
+                     stream);
 }
 
 }  // extern "C"

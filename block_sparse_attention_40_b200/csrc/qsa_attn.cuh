@@ -91,6 +91,7 @@ struct AttnArgs {
   int32_t decode;          // 1: decode (tile = sequence, KV from the block cache)
   int32_t splits;          // chunk splits per tile (decode), 1 for prefill
   int64_t cap_blocks;      // decode: capacity / 4
+  Paging pg;               // decode: where each sequence's K/V blocks live (table null: contiguous)
   __nv_bfloat16* out;      // prefill: [T][24][128]; decode with one split: [B][24][128]
   float* part_o;           // decode: [B][2][splits][12][128]
   float* part_m;           // decode: [B][2][splits][12]
@@ -124,21 +125,37 @@ __device__ __forceinline__ float ex2_approx(float x) {
 // (and the run of padding slots past the end of the union) are cut into power-of-two pieces;
 // the first lane of each run issues one TMA box per piece (rows 4*blk.., two 64-dim panels).
 // Run r of a chunk (in slot order) goes to warp r mod nw; warp 0 posts the chunk's bytes.
-// Padding rows come from an out-of-range coordinate and are zero-filled.
+// Padding rows come from an out-of-range coordinate and are zero-filled.  kPaged (a paged
+// decode cache): runs are also cut where a page starts, and each run's rows are looked up in
+// the page table of sequence seq (KV head g).  The other instances carry none of that code: the
+// prefill gather is limited by how fast these warps issue copies.
+template <bool kPaged>
 __device__ __forceinline__ void attn_producer(const CUtensorMap* maps, unsigned char* ring,
                                               uint64_t* full, uint64_t* empty, int stages,
                                               const int32_t* uni, int U, int c_begin, int nchunks,
                                               int64_t kv_row_base, int col0, int32_t oob_row,
+                                              const Paging& pg, int seq, int g,
                                               int w, int nw, volatile int* abort, DevStatus st,
                                               uint32_t site) {
   const int lane = threadIdx.x & 31;
   int upos = c_begin * AttnCfg::kChunkBlocks + lane;
   int blk_next = upos < U ? uni[upos] : -1;
+  // paged: the pool row of the slot's block, looked up a chunk ahead like the block itself
+  // (-1: out-of-range page entry); a piece of a run starts off blocks later in the same page
+  auto lookup = [&](int b) -> int64_t {
+    if constexpr (kPaged) return b >= 0 ? pool_kv_row(pg, seq, g, b) : 0;
+    return 0;
+  };
+  int64_t prow_next = lookup(blk_next);
   int issued = 0;
   for (int i = 0; i < nchunks; ++i) {
     const int blk = blk_next;           // -1: padding slot
+    const int64_t prow = prow_next;
     upos += AttnCfg::kChunkBlocks;
-    if (i + 1 < nchunks) blk_next = upos < U ? uni[upos] : -1;
+    if (i + 1 < nchunks) {
+      blk_next = upos < U ? uni[upos] : -1;
+      prow_next = lookup(blk_next);
+    }
     const int s = i % stages;
     bool ok = true;
     if (lane == 0) ok = mbar_wait(&empty[s], ((i / stages) & 1) ^ 1, abort, st, site);
@@ -147,7 +164,8 @@ __device__ __forceinline__ void attn_producer(const CUtensorMap* maps, unsigned 
     if (lane == 0 && w == 0) mbar_arrive_expect_tx(&full[s], AttnCfg::kKVBytes);
     __syncwarp();
     const int prev = __shfl_up_sync(0xffffffffu, blk, 1);
-    const bool start = lane == 0 || (blk < 0) != (prev < 0) || (blk >= 0 && blk != prev + 1);
+    bool start = lane == 0 || (blk < 0) != (prev < 0) || (blk >= 0 && blk != prev + 1);
+    if constexpr (kPaged) start = start || (blk >= 0 && blk % pg.page_blocks == 0);
     const unsigned starts = __ballot_sync(0xffffffffu, start);
     // (a box may complete before warp 0 posts the bytes: the phase cannot end while the
     // posting arrival is missing)
@@ -163,9 +181,15 @@ __device__ __forceinline__ void attn_producer(const CUtensorMap* maps, unsigned 
         const int lg_fit = 31 - __clz(rem);
         const int lg_align = slot == 0 ? 5 : __ffs(slot) - 1;
         const int lg = lg_fit < lg_align ? lg_fit : lg_align;
-        const int32_t row = blk < 0 ? oob_row
-                                    : static_cast<int32_t>(kv_row_base +
-                                                           static_cast<int64_t>(blk + off) * kBlock);
+        int32_t row = oob_row;
+        if (blk >= 0) {
+          if constexpr (kPaged) {
+            if (prow < 0) report_error(st, kErrDevice, 205);
+            else row = static_cast<int32_t>(prow + static_cast<int64_t>(off) * kBlock);
+          } else {
+            row = static_cast<int32_t>(kv_row_base + static_cast<int64_t>(blk + off) * kBlock);
+          }
+        }
         unsigned char* dst = ring + s * AttnCfg::kKVBytes + slot * 512;
         tma_load_2d(dst, &maps[lg], col0, row, &full[s]);
         tma_load_2d(dst + 16384, &maps[lg], col0 + 64, row, &full[s]);
@@ -181,8 +205,9 @@ __device__ __forceinline__ void attn_producer(const CUtensorMap* maps, unsigned 
   }
 }
 
-// kDec: decode layout (one query token per tile; see the decode softmax below).
-template <bool kDec>
+// kDec: decode layout (one query token per tile; see the decode softmax below).  kPaged: the
+// decode cache is paged (args.pg).
+template <bool kDec, bool kPaged = false>
 __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
     k_sparse_attn(const __grid_constant__ AttnMaps maps, AttnArgs args) {
   using C = AttnCfg;
@@ -328,8 +353,9 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
                       static_cast<int32_t>(tok_row0), q_full);
     }
     __syncwarp();
-    attn_producer(maps.k, sK, k_full, k_empty, C::kKStages, uni, U, c_begin, nchunks,
-                  kv_row_base, col0, args.oob_row, kw, C::kKWarps, s_abort, args.st, 20);
+    attn_producer<kPaged>(maps.k, sK, k_full, k_empty, C::kKStages, uni, U, c_begin, nchunks,
+                  kv_row_base, col0, args.oob_row, args.pg, tile, g, kw, C::kKWarps, s_abort,
+                  args.st, 20);
     if (kw == 0 && lane == 0 && *s_abort) mbar_drain(q_full, 0);
   } else if (warp >= C::kVWarp0) {
     // ---------------- V producers ----------------
@@ -337,8 +363,9 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
     if (vw == 0 && lane == 0)
       for (int j = 0; j < kNumBoxSizes; ++j) prefetch_tmap(&maps.v[j]);
     __syncwarp();
-    attn_producer(maps.v, sV, v_full, v_empty, C::kVStages, uni, U, c_begin, nchunks,
-                  kv_row_base, col0, args.oob_row, vw, C::kVWarps, s_abort, args.st, 27);
+    attn_producer<kPaged>(maps.v, sV, v_full, v_empty, C::kVStages, uni, U, c_begin, nchunks,
+                  kv_row_base, col0, args.oob_row, args.pg, tile, g, vw, C::kVWarps, s_abort,
+                  args.st, 27);
   } else {
     // ---------------- MMA issuer (warp kMmaWarp) ----------------
     if (lane == 0) {

@@ -51,6 +51,48 @@ __device__ __forceinline__ void report_error(DevStatus st, uint32_t code, uint32
 }
 
 // ----------------------------------------------------------------------------------------
+// Where a decode cache keeps its blocks.  Logical block blk of sequence b lives in pool page
+// table[b][blk / page_blocks], at block blk % page_blocks of that page; K/V rows are laid out
+// [pool page][KV head][page_blocks * 4 tokens], compressed keys [pool page][page_blocks].
+// A contiguous cache is the case table == nullptr: sequence b owns page b, which holds its
+// whole capacity (page_blocks = capacity / 4).
+struct Paging {
+  const int32_t* table;   // [batch][max_pages] or nullptr
+  int32_t max_pages;      // logical pages per sequence
+  int32_t page_blocks;    // blocks per page
+  int32_t pool_pages;     // pages in the pool
+};
+
+// Pool page of (b, blk) (-1 when the page table entry is out of range) and the block's index
+// inside it.  Block indices are below 2^18, so 32-bit arithmetic suffices.
+__device__ __forceinline__ int32_t pool_page(const Paging& pg, int b, int64_t blk, int32_t* in) {
+  if (pg.table == nullptr) {
+    *in = static_cast<int32_t>(blk);
+    return b;
+  }
+  const int32_t lp = static_cast<int32_t>(blk) / pg.page_blocks;
+  *in = static_cast<int32_t>(blk) - lp * pg.page_blocks;
+  const int32_t page = pg.table[static_cast<int64_t>(b) * pg.max_pages + lp];
+  return (page < 0 || page >= pg.pool_pages) ? -1 : page;
+}
+
+// Pool block index of (b, blk), or -1 when the page table entry is out of range.
+__device__ __forceinline__ int64_t pool_block(const Paging& pg, int b, int64_t blk) {
+  int32_t in;
+  const int32_t page = pool_page(pg, b, blk, &in);
+  return page < 0 ? -1 : static_cast<int64_t>(page) * pg.page_blocks + in;
+}
+
+// First of the 4 K/V rows of (b, KV head g, blk), or -1 when the page table entry is out of
+// range.
+__device__ __forceinline__ int64_t pool_kv_row(const Paging& pg, int b, int g, int64_t blk) {
+  int32_t in;
+  const int32_t page = pool_page(pg, b, blk, &in);
+  if (page < 0) return -1;
+  return ((static_cast<int64_t>(page) * 2 + g) * pg.page_blocks + in) * kBlock;
+}
+
+// ----------------------------------------------------------------------------------------
 // Small PTX helpers.
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

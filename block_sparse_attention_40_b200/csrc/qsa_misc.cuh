@@ -199,11 +199,12 @@ struct AppendParams {
   int32_t n_new;
   int32_t batch;
   int32_t capacity;
-  uint4* k_blocks;     // [B][2][cap/4][4][128]
+  uint4* k_blocks;     // [pool pages][2][page blocks][4][128] (contiguous: [B][2][cap/4][4][128])
   uint4* v_blocks;
-  uint4* kbar;         // [B][cap/4][64]
+  uint4* kbar;         // [pool pages][page blocks][64] (contiguous: [B][cap/4][64])
   float* partial;      // [B][64]
   const int32_t* len;  // [B]
+  Paging pg;
   DevStatus st;
 };
 
@@ -215,7 +216,6 @@ __device__ __forceinline__ int append_count(const AppendParams& p, int b) {
 // Copies: one work item per 16 bytes of K and V (items 0 .. batch * n_new * 32).
 __device__ __forceinline__ void append_copy_item(const AppendParams& p, int64_t i) {
   const int64_t per_tok = 2 * 16;                       // 2 heads x 16 units of 16 B
-  const int64_t cap_blk = p.capacity / kBlock;
   {
     const int b = static_cast<int>(i / (static_cast<int64_t>(p.n_new) * per_tok));
     const int64_t rem = i - static_cast<int64_t>(b) * p.n_new * per_tok;
@@ -228,8 +228,12 @@ __device__ __forceinline__ void append_copy_item(const AppendParams& p, int64_t 
       report_error(p.st, kErrDevice, 200);
       return;
     }
-    const int64_t dst = ((((static_cast<int64_t>(b) * 2 + g) * cap_blk + pos / 4) * 4 + pos % 4) *
-                         16) + u;
+    const int64_t row0 = pool_kv_row(p.pg, b, g, pos / 4);   // the block's first row
+    if (row0 < 0) {
+      report_error(p.st, kErrDevice, 202);
+      return;
+    }
+    const int64_t dst = (row0 + pos % 4) * 16 + u;
     const int64_t src = ((static_cast<int64_t>(b) * p.n_new + j) * 2 + g) * 16 + u;
     p.k_blocks[dst] = p.k[src];
     p.v_blocks[dst] = p.v[src];
@@ -237,8 +241,7 @@ __device__ __forceinline__ void append_copy_item(const AppendParams& p, int64_t 
     // yet written are finite (attention reads whole blocks and masks the future rows).
     if (j == append_count(p, b) - 1) {
       for (int64_t q = pos + 1; q < (pos / 4) * 4 + 4; ++q) {
-        const int64_t dz = ((((static_cast<int64_t>(b) * 2 + g) * cap_blk + q / 4) * 4 + q % 4) *
-                            16) + u;
+        const int64_t dz = (row0 + q % 4) * 16 + u;
         p.k_blocks[dz] = make_uint4(0, 0, 0, 0);
         p.v_blocks[dz] = make_uint4(0, 0, 0, 0);
       }
@@ -252,7 +255,6 @@ __device__ __forceinline__ void append_copy_item(const AppendParams& p, int64_t 
 __device__ __forceinline__ void append_kbar_item(const AppendParams& p, int64_t i,
                                                  int max_blocks_touched) {
   const int64_t slots = static_cast<int64_t>(max_blocks_touched);
-  const int64_t cap_blk = p.capacity / kBlock;
   {
     const int b = static_cast<int>(i / (slots * 8));
     const int64_t slot = (i / 8) % slots;
@@ -268,7 +270,7 @@ __device__ __forceinline__ void append_kbar_item(const AppendParams& p, int64_t 
     const int64_t jf = L0 / 4, jl = (L1 - 1) / 4;
     const uint4* kin = p.k_idx + static_cast<int64_t>(b) * p.n_new * 8 + part;  // token j at +8j
     float* part_sum = p.partial + static_cast<int64_t>(b) * 64 + part * 8;
-    uint4* kb_out = p.kbar + (static_cast<int64_t>(b) * cap_blk) * 8 + part;
+    uint4* kb_out = p.kbar + part;   // + 8 x the pool block
     auto add_tokens = [&](float* acc, int64_t from, int64_t to, bool start_from_first) {
       // sum tokens [from, to) (absolute positions) into acc in order
       for (int64_t pos = from; pos < to; ++pos) {
@@ -294,7 +296,12 @@ __device__ __forceinline__ void append_kbar_item(const AppendParams& p, int64_t 
 #pragma unroll
         for (int q = 0; q < 4; ++q)
           po[q] = pack_bf16x2(__fmul_rn(acc[2 * q], 0.25f), __fmul_rn(acc[2 * q + 1], 0.25f));
-        kb_out[j * 8] = o;
+        const int64_t pb = pool_block(p.pg, b, j);
+        if (pb < 0) {
+          report_error(p.st, kErrDevice, 203);
+          return;
+        }
+        kb_out[pb * 8] = o;
       } else {
 #pragma unroll
         for (int q = 0; q < 8; ++q) part_sum[q] = acc[q];

@@ -59,6 +59,8 @@ struct ScoreArgs {
   int32_t splits;
   int32_t mtiles_per_split;
   int64_t kbar_rows_per_seq;
+  Paging pg;               // where each sequence's compressed keys live (table null: contiguous)
+  int32_t kbar_oob_row;    // a row past the compressed-key pool (TMA reads it as zeros)
   int32_t* n_c_out;        // [B] n_c per sequence (written by split 0), may be null
   uint32_t* hist;          // [B][4096] first-digit histograms of the scores (zeroed), or null
   // common
@@ -77,6 +79,7 @@ struct ScoreWork {
   int32_t ntok;      // valid tokens in the N tile
   int32_t pos0;      // position (within the sequence) of token 0
   int64_t out_row0;  // score row of token 0
+  int32_t seq;       // decode: the sequence
 };
 
 // s = sum_h w[h] * ReLU(d[h]) over the 16 heads of one (token, block): the even and the odd
@@ -122,6 +125,7 @@ __device__ __forceinline__ ScoreWork<NTOK> score_work(const ScoreArgs& a) {
     wk.a_row0 = m.kbar0;
     wk.b_row0 = static_cast<int32_t>((m.tok0 + p0) * kIdxHeads);
     wk.out_row0 = m.tok0 + p0 - a.row_begin;
+    wk.seq = s;
   } else {
     const int b = static_cast<int>(blockIdx.x) / a.splits;
     const int split = static_cast<int>(blockIdx.x) % a.splits;
@@ -139,6 +143,7 @@ __device__ __forceinline__ ScoreWork<NTOK> score_work(const ScoreArgs& a) {
     wk.a_row0 = static_cast<int64_t>(b) * a.kbar_rows_per_seq;
     wk.b_row0 = b * kIdxHeads;
     wk.out_row0 = b;
+    wk.seq = b;
   }
   return wk;
 }
@@ -218,12 +223,26 @@ __global__ void __launch_bounds__(ScoreCfg<NTOK>::kThreads, ScoreCfg<NTOK>::kCta
       mbar_arrive_expect_tx(b_full, C::kBBytes);
       tma_load_2d(sB, &tmap_qidx, 0, wk.b_row0, b_full);
       int issued = 0;
+      // row of M-tile m's first compressed key; paged caches look the page up (an M-tile of
+      // 128 blocks lies inside one page), one tile ahead of its copy
+      auto tile_row = [&](int m) -> int64_t {
+        if constexpr (NTOK == 1) {
+          if (args.pg.table != nullptr) {
+            const int64_t r = pool_block(args.pg, wk.seq, 128ll * m);
+            if (r < 0) report_error(args.st, kErrDevice, 204);
+            return r < 0 ? static_cast<int64_t>(args.kbar_oob_row) : r;
+          }
+        }
+        return wk.a_row0 + 128ll * m;
+      };
+      int64_t row_next = wk.n_mtiles > 0 ? tile_row(wk.mt0) : 0;
       for (int i = 0; i < wk.n_mtiles; ++i) {
         const int s = i % C::kStages;
+        const int64_t row = row_next;
+        if (i + 1 < wk.n_mtiles) row_next = tile_row(wk.mt0 + i + 1);
         if (!mbar_wait(&empty[s], ((i / C::kStages) & 1) ^ 1, s_abort, args.st, 10)) break;
         mbar_arrive_expect_tx(&full[s], C::kABytes);
-        tma_load_2d(sA + s * C::kABytes, &tmap_kbar, 0,
-                    static_cast<int32_t>(wk.a_row0 + 128ll * (wk.mt0 + i)), &full[s]);
+        tma_load_2d(sA + s * C::kABytes, &tmap_kbar, 0, static_cast<int32_t>(row), &full[s]);
         ++issued;
       }
       if (*s_abort) {

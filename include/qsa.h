@@ -252,6 +252,47 @@ QSA_API qsa_status qsa_decode_noalloc(const void *q, const qsa_cache *cache, con
                                       int32_t *sel_idx, int32_t *sel_cnt, qsa_params params,
                                       qsa_stream_t stream);
 
+/* ---------------------------------------------------------------------------------- */
+/* Paged KV cache (aiany.app "Qwen3.8-Flash-Next", "Implementation notes": the model ships
+ * with serving recipes for vLLM and SGLang, and KV cache sizing for very long contexts is
+ * an operational concern).  Those frameworks keep their caches in pages; the pages give no
+ * page layout, so the one below is this library's own.  Sequences own fixed-size pages of
+ * one shared pool, listed in a page table, so that a batch of sequences of very different
+ * lengths needs pool memory only for the pages it has reached:
+ *   base.k_blocks, base.v_blocks : bf16 [pool_pages][2][page_tokens/4][4][128]
+ *   base.kbar                    : bf16 [pool_pages][page_tokens/4][64]
+ *   base.kbar_partial, base.len  : per sequence, as in qsa_cache
+ *   page_table : int32 [batch][base.capacity/page_tokens] device: logical page j of sequence
+ *                b (its tokens j*page_tokens ..) lives in pool page page_table[b][j]
+ * base.capacity is the logical capacity per sequence, a multiple of page_tokens; page_tokens
+ * is a multiple of 512 (an indexer tile of 128 blocks then never spans two pages), and
+ * pool_pages * 2 * page_tokens < 2^31.  Only the entries of pages a sequence has reached are
+ * read.  Each must lie in 0 .. pool_pages-1, and live sequences must not share a page.  An
+ * entry out of range is never followed: the append skips the writes that would go there
+ * (it has no workspace to report in), and the decode reads zeros there and records
+ * QSA_ERR_DEVICE.  Same arguments, results and errors as qsa_append_kv, qsa_decode and
+ * qsa_decode_workspace_size otherwise (the workspace size is the contiguous cache's); the
+ * results are bit-identical to those of a contiguous cache holding the same tokens. */
+typedef struct {
+  qsa_cache base;
+  int32_t *page_table;
+  int32_t page_tokens;
+  int32_t pool_pages;
+} qsa_paged_cache;
+
+QSA_API qsa_status qsa_append_kv_paged(const qsa_paged_cache *cache, const void *k,
+                                       const void *v, const void *k_idx, int32_t n_new,
+                                       const int32_t *counts, const int32_t *h_len,
+                                       qsa_stream_t stream);
+
+QSA_API size_t qsa_decode_paged_workspace_size(const qsa_paged_cache *cache, qsa_params params);
+
+QSA_API qsa_status qsa_decode_paged(const void *q, const qsa_paged_cache *cache,
+                                    const void *q_idx, const void *w, void *out,
+                                    const int32_t *h_len, int32_t *sel_idx, int32_t *sel_cnt,
+                                    void *workspace, size_t ws_bytes, qsa_params params,
+                                    qsa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

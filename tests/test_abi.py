@@ -106,3 +106,36 @@ def test_cpu_tensors_are_refused():
     q = torch.zeros((8, 24, 128), dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):
         B._need(q, "q", torch.bfloat16, (24, 128), 3)
+
+
+def test_paged_cache_host_side_checks():
+    lib = qsa.load()
+    good = 0x10000
+    prm = B._params(512)
+
+    def paged(page_tokens=4096, pool=200, cap=262144, batch=64, table=good):
+        return B.PagedCacheDesc(B.CacheDesc(good, good, good, good, good, batch, cap), table,
+                                page_tokens, pool)
+
+    base = B.CacheDesc(good, good, good, good, good, 64, 262144)
+    n = lib.qsa_decode_paged_workspace_size(ctypes.byref(paged()), prm)
+    assert n == lib.qsa_decode_workspace_size(ctypes.byref(base), prm) > 0
+    for bad in (paged(page_tokens=1000), paged(page_tokens=0), paged(cap=262144 + 512),
+                paged(pool=0), paged(table=0), paged(pool=1 << 20)):
+        assert lib.qsa_decode_paged_workspace_size(ctypes.byref(bad), prm) == 0
+    h_len = (ctypes.c_int32 * 2)(60, 10)
+    r = lib.qsa_append_kv_paged(ctypes.byref(paged(batch=2, cap=1024, page_tokens=512)), _p(good),
+                                _p(good), _p(good), 1000, None, h_len, None)
+    assert B.STATUS[r] == "QSA_ERR_CAPACITY"
+    r = lib.qsa_append_kv_paged(ctypes.byref(paged(batch=2, cap=1024, page_tokens=1000)),
+                                _p(good), _p(good), _p(good), 8, None, h_len, None)
+    assert B.STATUS[r] == "QSA_ERR_INVALID_ARG"
+    r = lib.qsa_append_kv_paged(ctypes.byref(paged(batch=2, cap=1024, page_tokens=512,
+                                                   table=good + 2)),
+                                _p(good), _p(good), _p(good), 8, None, h_len, None)
+    assert B.STATUS[r] == "QSA_ERR_ALIGNMENT"
+    h_len = (ctypes.c_int32 * 2)(0, 10)
+    r = lib.qsa_decode_paged(_p(good), ctypes.byref(paged(batch=2, cap=1024, page_tokens=512)),
+                             _p(good), _p(good), _p(good), h_len, None, None, _p(good), 1 << 30,
+                             B._params(16), None)
+    assert B.STATUS[r] == "QSA_ERR_INVALID_ARG"

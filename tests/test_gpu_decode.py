@@ -33,14 +33,16 @@ def _oracle_row(k_tok, v_tok, kidx_tok, q, q_idx, w, topk, forced=None):
 
 
 def _decode_session(spec, check_seqs, steps, splits=0, device_gen=False, ctx_fn=None,
-                    step_fn=None, exact_sel=False):
+                    step_fn=None, exact_sel=False, cache_fn=None):
     """ctx_fn(k, v, k_idx) and step_fn(step dict) may reshape the seeded inputs (ties);
-    exact_sel demands the oracle's selection itself (inputs whose scores are exact)."""
+    exact_sel demands the oracle's selection itself (inputs whose scores are exact);
+    cache_fn(spec) builds the cache (default: a contiguous KVCache)."""
     gen_dev = DEV if device_gen else "cpu"
     k_ctx, v_ctx, ki_ctx = W.decode_context(spec, device=gen_dev)
     if ctx_fn is not None:
         k_ctx, v_ctx, ki_ctx = ctx_fn(k_ctx, v_ctx, ki_ctx)
-    cache = qsa.KVCache(spec.batch, spec.capacity, DEV, zero=False)
+    cache = (cache_fn(spec) if cache_fn is not None
+             else qsa.KVCache(spec.batch, spec.capacity, DEV, zero=False))
     # bulk fill in chunks with per-sequence counts
     lmax = max(spec.context)
     chunk = 16384
@@ -87,7 +89,8 @@ def _decode_session(spec, check_seqs, steps, splits=0, device_gen=False, ctx_fn=
             results.append((b, step, swaps) + compare_outputs(out[b:b + 1], o_out))
             # the compressed cache agrees bit for bit with the oracle's compression
             L = kt.shape[0]
-            got = cache.kbar[b, :L // 4].contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+            got = cache.kbar_rows(b, L // 4).contiguous().cpu().view(torch.int16).numpy().view(
+                np.uint16)
             assert np.array_equal(got, kbar[:L // 4])
     return results
 
