@@ -457,7 +457,7 @@ def main():
                             # capture of the 32K prefill (profiles/k_sparse_attn_prefill_32k.md),
                             # scaled by tokens (the traffic is q, the plan and the output; K/V
                             # stay in L2)
-                            "traffic": 489.999e6 * args.prefill_len / 32768,
+                            "traffic": 489.548e6 * args.prefill_len / 32768,
                             "traffic_source": "ncu capture at 32K, scaled by tokens",
                             "algorithmic": f"{attn_flops / 1e12:.4f} TFLOP selected-token per launch"}
         idx_flops = prefill_indexer_flops(args.prefill_len)
