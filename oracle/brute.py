@@ -118,3 +118,25 @@ def run_sequence(q, k, v, q_idx, k_idx, w, topk, rows=None):
         tokens = [4 * b + j for b in sel for j in range(B)] + list(range(4 * c, t + 1))
         res[t] = (sel, attend(q[t], k, v, tokens) if q is not None else None)
     return res, kbar
+
+
+def kth_ranked_score(scores, k):
+    """Score of the candidate ranked k-th (exactly k-1 candidates beat it: a higher score,
+    or an equal score at a lower index), or None when there are at most k candidates and
+    nothing is left out.  This is the selection boundary: the lowest kept score."""
+    n = len(scores)
+    if n <= k:
+        return None
+    for b in range(n):
+        beaten_by = sum(1 for c in range(n)
+                        if scores[c] > scores[b] or (scores[c] == scores[b] and c < b))
+        if beaten_by == k - 1:
+            return scores[b]
+    raise AssertionError("no candidate has rank k")
+
+
+def row_scores(q_idx, k_idx, w, rows):
+    """{t: [s(t, b) for every candidate block b < floor(t/4)]} for ONE sequence (nested
+    lists of floats, token-major)."""
+    kbar = compress_seq(k_idx)
+    return {t: [score(q_idx[t], w[t], kbar[b]) for b in range(t // B)] for t in rows}

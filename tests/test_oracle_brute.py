@@ -57,3 +57,30 @@ def test_brute_needles():
     p = W.custom_prefill([48], topk=2, kind="needle", seed=9, needles_per_seq=2,
                          needle_range=(1, 10))
     _check(p, rows_attn={47})
+
+
+@pytest.mark.parametrize("seed,kind,topk", [(3, "normal", 3), (4, "normal", 5), (6, "int", 2)])
+def test_kth_is_the_boundary_score(seed, kind, topk):
+    # The oracle reports, per row, the score of its last kept block: the anchor of the
+    # tie band within which a GPU selection may swap blocks.  The brute force finds the
+    # same value by rank counting; rows with at most k candidates report -1 (no boundary).
+    p = W.custom_prefill([45], topk=topk, kind=kind, seed=seed)
+    b = prefill_bits(p)
+    idx, cnt, kth, _, _ = oracle.prefill(q=None, k=b["k"], v=b["v"], q_idx=b["q_idx"],
+                                         k_idx=b["k_idx"], w=b["w"], cu_seqlens=b["cu_seqlens"],
+                                         topk=topk)
+    sc = brute.row_scores(to_lists(p.q_idx), to_lists(p.k_idx), to_lists(p.w), range(45))
+    bounded = 0
+    for t in range(45):
+        want = brute.kth_ranked_score(sc[t], topk)
+        if want is None:
+            assert kth[t] == -1.0, (t, kth[t])
+        else:
+            assert abs(kth[t] - want) <= 1e-12 * max(1.0, abs(want)), (t, kth[t], want)
+            # the boundary is the lowest kept score and no dropped block beats it
+            kept = set(idx[t, :cnt[t]].tolist())
+            assert min(sc[t][x] for x in kept) == pytest.approx(want, rel=1e-12, abs=1e-12)
+            assert all(sc[t][x] <= want + 1e-12 * max(1.0, abs(want))
+                       for x in range(len(sc[t])) if x not in kept)
+            bounded += 1
+    assert bounded >= 20

@@ -160,3 +160,42 @@ def test_8k_needles_sampled_rows():
     for i, t in enumerate(rows):
         sel = set(idx[i, :cnt[i]].tolist())
         assert {n for n in p.needles[0] if n < t // 4} <= sel
+
+
+def test_forced_own_selection_reproduces_outputs():
+    # Handing the oracle its own selection through the forced path changes nothing: the
+    # forced path attends exactly the blocks it is given (the GPU parity tests compare
+    # outputs through this path, on the GPU's selection).
+    p = W.custom_prefill([97, 66], topk=5, kind="normal", seed=14)
+    idx, cnt, _, out, _ = _run(p)
+    b = prefill_bits(p)
+    _, _, _, out_f, _ = oracle.prefill(q=b["q"], k=b["k"], v=b["v"], q_idx=b["q_idx"],
+                                       k_idx=b["k_idx"], w=b["w"], cu_seqlens=b["cu_seqlens"],
+                                       topk=p.topk, forced_idx=idx, forced_cnt=cnt)
+    assert np.array_equal(out_f, out)
+
+
+def test_forced_selection_attends_exactly_the_given_blocks():
+    # Arbitrary forced selections (seeded random ascending subsets of the candidates, of
+    # any size up to k, including empty ones and dense prefixes) give dense attention
+    # under the mask those blocks plus the own block make: fp64 SDPA, a library routine.
+    T, k = 150, 9
+    p = W.custom_prefill([T], topk=k, kind="normal", seed=15)
+    rng = np.random.default_rng(15)
+    fi = np.full((T, k), -1, dtype=np.int32)
+    fc = np.zeros(T, dtype=np.int32)
+    for t in range(T):
+        n_c = t // 4
+        if t % 5 == 0:
+            sel = np.arange(min(k, n_c))                       # a dense prefix
+        else:
+            m = int(rng.integers(0, min(k, n_c) + 1))
+            sel = np.sort(rng.choice(n_c, size=m, replace=False)) if m else np.zeros(0, int)
+        fi[t, :len(sel)] = sel
+        fc[t] = len(sel)
+    b = prefill_bits(p)
+    _, _, _, out, _ = oracle.prefill(q=b["q"], k=b["k"], v=b["v"], q_idx=b["q_idx"],
+                                     k_idx=b["k_idx"], w=b["w"], cu_seqlens=b["cu_seqlens"],
+                                     topk=k, forced_idx=fi, forced_cnt=fc)
+    ref = dense_gqa_reference(p.q, p.k, p.v, _mask_from_selection(T, fi, fc))
+    np.testing.assert_allclose(out, ref.numpy(), rtol=0, atol=1e-12)

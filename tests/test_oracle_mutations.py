@@ -38,6 +38,15 @@ MUTANTS = {
                        "tests/test_oracle_compress.py::test_order_sensitive_inputs_match_torch_fp32"),
     "score_weight_dropped": ("s += bf(w[h]) * r;", "s += r;",
                              "tests/test_oracle_brute.py::test_brute_random"),
+    "kth_off_by_one": ("*kth = c[k - 1].s;", "*kth = c[k].s;",
+                       "tests/test_oracle_brute.py::test_kth_is_the_boundary_score"),
+    "kth_sentinel": ("*kth = -1.0;", "*kth = 0.0;",
+                     "tests/test_oracle_brute.py::test_kth_is_the_boundary_score"),
+    "forced_row_ignored": ("idx = (int32_t *)(forced_idx + r * topk);",
+                           "idx = (int32_t *)(forced_idx);",
+                           "tests/test_oracle_invariants.py::test_forced_selection_attends_exactly_the_given_blocks"),
+    "forced_count_short": ("cnt = forced_cnt[r];", "cnt = forced_cnt[r] > 0 ? forced_cnt[r] - 1 : 0;",
+                           "tests/test_oracle_invariants.py::test_forced_own_selection_reproduces_outputs"),
 }
 
 
