@@ -35,6 +35,35 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 PREFILL_T, TOPK = 65536, 512
 DEC_BATCH, DEC_CAP = 64, 262144
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the roofline kernels from one
+# ncu capture: bytes per unit of work (prefill attention: per query token; decode step: per
+# sequence), the SHA-256 of the kernel sources the capture ran, and what was captured.  A
+# figure is reported only while the sources are unchanged; otherwise the roofline's
+# "traffic" is null until a new capture is taken.
+NCU_TRAFFIC = {}
+
+
+def csrc_sha():
+    import hashlib
+    d = os.path.join(ROOT, "block_sparse_attention_40_b200", "csrc")
+    h = hashlib.sha256()
+    for n in sorted(os.listdir(d)):
+        if n.endswith((".cu", ".cuh")):
+            h.update(n.encode())
+            h.update(open(os.path.join(d, n), "rb").read())
+    return h.hexdigest()
+
+
+def measured_traffic(kernel, units):
+    """Per-launch DRAM bytes of `kernel` scaled to `units`, or (None, reason)."""
+    rec = NCU_TRAFFIC.get(kernel)
+    if rec is None:
+        return None, "no ncu capture of the current kernel"
+    per_unit, sha, what = rec
+    if sha != csrc_sha():
+        return None, "kernel sources changed since the ncu capture"
+    return per_unit * units, what
+
 
 # ------------------------------------------------------------------------------------
 # algorithmic work (definitions; the kernels never read these)
@@ -453,13 +482,10 @@ def main():
                             "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
                             "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
                             "peak_source": f"{r['peak_src']} bf16 burst",
-                            # dram__bytes_read + dram__bytes_write of this kernel from one ncu
-                            # capture of the 32K prefill (profiles/k_sparse_attn_prefill_32k.md),
-                            # scaled by tokens (the traffic is q, the plan and the output; K/V
-                            # stay in L2)
-                            "traffic": 489.548e6 * args.prefill_len / 32768,
-                            "traffic_source": "ncu capture at 32K, scaled by tokens",
+                            "traffic": None, "traffic_source": None,
                             "algorithmic": f"{attn_flops / 1e12:.4f} TFLOP selected-token per launch"}
+        line["roofline"]["traffic"], line["roofline"]["traffic_source"] = measured_traffic(
+            "prefill_attention", args.prefill_len)
         idx_flops = prefill_indexer_flops(args.prefill_len)
         line["prefill"] = {"tokens_per_s": world * args.prefill_len / (pre_ms / 1e3),
                            "ms": pre_ms, "select_ms": r["sel_ms"] / K, "attention_ms": r["att_ms"] / K,
@@ -477,8 +503,10 @@ def main():
                             "peak": peaks["hbm_gbs"], "unit": "GB/s",
                             "frac": gbs / peaks["hbm_gbs"],
                             "peak_source": f"{r['peak_src']} HBM copy",
-                            "traffic": None,
+                            "traffic": None, "traffic_source": None,
                             "algorithmic": f"{r['dec_bytes'] / 1e6:.1f} MB per step"}}
+        dec["roofline"]["traffic"], dec["roofline"]["traffic_source"] = measured_traffic(
+            "decode_step", args.decode_batch)
         if "decode" in r["e2e"]:
             dec["e2e"] = r["e2e"]["decode"]
         line["decode"] = dec

@@ -30,8 +30,8 @@ EXPORTS = ("qsa_status_string", "qsa_version", "qsa_launch_count", "qsa_workspac
            "qsa_compress_workspace_size", "qsa_compress", "qsa_index_scores", "qsa_topk",
            "qsa_prefill_workspace_size", "qsa_prefill", "qsa_prefill_select",
            "qsa_sparse_attention", "qsa_append_kv", "qsa_decode_workspace_size", "qsa_decode",
-           "qsa_decode_noalloc", "qsa_append_kv_paged", "qsa_decode_paged_workspace_size",
-           "qsa_decode_paged")
+           "qsa_decode_noalloc", "qsa_noalloc_last_device_error", "qsa_append_kv_paged",
+           "qsa_decode_paged_workspace_size", "qsa_decode_paged")
 
 
 class QSAError(RuntimeError):
@@ -42,7 +42,8 @@ class QSAError(RuntimeError):
 
 class Params(ctypes.Structure):
     _fields_ = [("topk_blocks", ctypes.c_int32), ("rows_per_tile", ctypes.c_int32),
-                ("decode_splits", ctypes.c_int32), ("score_chunk_rows", ctypes.c_int32)]
+                ("decode_splits", ctypes.c_int32), ("score_chunk_rows", ctypes.c_int32),
+                ("debug_fault", ctypes.c_int32)]
 
 
 class CacheDesc(ctypes.Structure):
@@ -92,6 +93,7 @@ def load(build_if_needed: bool = True):
             "qsa_decode_workspace_size": ([P, Params], SZ),
             "qsa_decode": ([P, P, P, P, P, P, P, P, P, SZ, Params, P], st),
             "qsa_decode_noalloc": ([P, P, P, P, P, P, P, P, Params, P], st),
+            "qsa_noalloc_last_device_error": ([P, P], st),
             "qsa_append_kv_paged": ([P, P, P, P, I32, P, P, P], st),
             "qsa_decode_paged_workspace_size": ([P, Params], SZ),
             "qsa_decode_paged": ([P, P, P, P, P, P, P, P, P, SZ, Params, P], st),
@@ -147,8 +149,9 @@ def _cu_pair(cu_seqlens, device):
     return h, d
 
 
-def _params(topk, rows_per_tile=0, decode_splits=0, score_chunk_rows=0) -> Params:
-    return Params(int(topk), int(rows_per_tile), int(decode_splits), int(score_chunk_rows))
+def _params(topk, rows_per_tile=0, decode_splits=0, score_chunk_rows=0, debug_fault=0) -> Params:
+    return Params(int(topk), int(rows_per_tile), int(decode_splits), int(score_chunk_rows),
+                  int(debug_fault))
 
 
 def new_workspace(nbytes: int, device) -> torch.Tensor:
@@ -268,12 +271,13 @@ def topk(scores: torch.Tensor, n_c: torch.Tensor, k: int, max_n_c: Optional[int]
 class Prefill:
     """Reusable prefill context: holds the device cu_seqlens and the workspace."""
 
-    def __init__(self, cu_seqlens, device, topk=512, rows_per_tile=0, score_chunk_rows=0):
+    def __init__(self, cu_seqlens, device, topk=512, rows_per_tile=0, score_chunk_rows=0,
+                 debug_fault=0):
         self.device = torch.device(device)
         self.h_cu, self.d_cu = _cu_pair(cu_seqlens, self.device)
         self.num_seqs = self.h_cu.numel() - 1
         self.T = int(self.h_cu[-1])
-        self.params = _params(topk, rows_per_tile, 0, score_chunk_rows)
+        self.params = _params(topk, rows_per_tile, 0, score_chunk_rows, debug_fault)
         self.topk = int(topk)
         self.ws = new_workspace(prefill_workspace_size(self.h_cu, topk, rows_per_tile,
                                                        score_chunk_rows), self.device)
@@ -494,3 +498,11 @@ def decode_noalloc(cache: KVCache, q, q_idx, w, topk=512, decode_splits=0, out=N
         _ptr(q), ctypes.byref(desc), _ptr(q_idx), _ptr(w), _ptr(out), h_len, None, None,
         _params(topk, 0, decode_splits, 0), _stream(q.device)))
     return out
+
+
+def noalloc_device_error(device) -> tuple:
+    """(status name, site) of the last decode_noalloc call, read from the library's own
+    scratch (synchronises the current stream of `device`)."""
+    site = ctypes.c_uint32(0)
+    code = load().qsa_noalloc_last_device_error(_stream(torch.device(device)), ctypes.byref(site))
+    return STATUS.get(code, str(code)), int(site.value)

@@ -98,6 +98,7 @@ struct PrefillGeom {
   int32_t R = kDefaultRowsPerTile;
   int32_t topk = 512;
   int32_t chunk_rows = kDefaultScoreChunkRows;
+  int32_t fault = 0;   // qsa_params.debug_fault
   PlanLayout pl;
   int32_t max_words = 1;
   // workspace offsets
@@ -108,7 +109,9 @@ qsa_status prefill_geom(const int32_t* h_cu, int32_t num_seqs, const qsa_params&
                         PrefillGeom* g) {
   if (!h_cu || num_seqs <= 0) return QSA_ERR_INVALID_ARG;
   if (p.topk_blocks < 1 || p.topk_blocks > QSA_MAX_TOPK) return QSA_ERR_INVALID_ARG;
+  if (p.debug_fault != 0 && p.debug_fault != 1) return QSA_ERR_INVALID_ARG;
   if (h_cu[0] != 0) return QSA_ERR_INVALID_ARG;
+  g->fault = p.debug_fault;
   g->R = p.rows_per_tile > 0 ? p.rows_per_tile : kDefaultRowsPerTile;
   if (g->R < 1 || g->R > 10) return QSA_ERR_INVALID_ARG;
   g->topk = p.topk_blocks;
@@ -366,6 +369,7 @@ qsa_status run_attention(const void* q, const void* k, const void* v, const int3
   a.splits = 1;
   a.out = reinterpret_cast<__nv_bfloat16*>(out);
   a.st = dev_status(ws);
+  a.fault_tile = g.fault == 1 ? g.attn_tiles - 1 : -1;
   dim3 grid(g.attn_tiles, 2, 1);
   k_sparse_attn<false><<<grid, AttnCfg::kThreads, AttnCfg::kSmemBytes, s>>>(maps, a);
   QSA_CHECK_LAUNCH();
@@ -438,6 +442,7 @@ qsa_status decode_geom(const qsa_cache* c, const qsa_params& p, DecodeGeom* g) {
       c->capacity > QSA_MAX_SEQ_LEN)
     return QSA_ERR_INVALID_ARG;
   if (p.topk_blocks < 1 || p.topk_blocks > QSA_MAX_TOPK) return QSA_ERR_INVALID_ARG;
+  if (p.debug_fault != 0) return QSA_ERR_INVALID_ARG;   // the fault hook is prefill-only
   g->B = c->batch;
   g->cap = c->capacity;
   g->topk = p.topk_blocks;
@@ -910,6 +915,7 @@ qsa_status decode_impl(const void* q, const CacheView& view, const void* q_idx, 
     a.part_m = reinterpret_cast<float*>(ws + g.o_pm);
     a.part_l = reinterpret_cast<float*>(ws + g.o_pl);
     a.st = dev_status(ws);
+    a.fault_tile = -1;
     dim3 grid(g.B, 2, g.splits);
     a.out = reinterpret_cast<__nv_bfloat16*>(out);   // written directly with one split
     if (view.pg.table != nullptr) {
@@ -958,7 +964,7 @@ qsa_status qsa_decode_paged(const void* q, const qsa_paged_cache* cache, const v
 // ---- decode with the library's own fixed scratch -----------------------------------------
 // One device array per GPU that loads the library, used as the workspace of
 // qsa_decode_noalloc.  In host code its name only stands for the symbol; the device
-// address comes from cudaGetSymbolAddress, looked up once per device with it current.
+// address comes from cudaGetSymbolAddress with the device current.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[QSA_NOALLOC_SCRATCH_BYTES];
 
 namespace {
@@ -966,14 +972,22 @@ constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[kMaxDevices] = {};
 
-qsa_status noalloc_scratch(void** out) {
+// The array's address on the current device.  It is looked up again on every call made
+// outside a stream capture (so that a module reloaded after cudaDeviceReset is followed);
+// during a capture the address of the last uncaptured call on this device is used, since a
+// capture must not call into the runtime for the symbol (make one call before capturing).
+qsa_status noalloc_scratch(cudaStream_t s, void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QSA_ERR_CUDA;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) return QSA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  if (cs == cudaStreamCaptureStatusNone) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return QSA_ERR_CUDA;
     g_noalloc_ptr[dev] = p;
+  } else if (!g_noalloc_ptr[dev]) {
+    return QSA_ERR_CUDA;   // no uncaptured call yet on this device
   }
   *out = g_noalloc_ptr[dev];
   return QSA_OK;
@@ -994,13 +1008,31 @@ extern "C" qsa_status qsa_decode_noalloc(const void* q, const qsa_cache* cache, 
             need, static_cast<unsigned>(QSA_NOALLOC_SCRATCH_BYTES));
     return QSA_ERR_WORKSPACE;
   }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   void* ws = nullptr;
-  qsa_status st = noalloc_scratch(&ws);
+  qsa_status st = noalloc_scratch(s, &ws);
   if (st != QSA_OK) return st;
   // the status words must start at zero; everything else is written before it is read
-  if (cudaMemsetAsync(ws, 0, QSA_WS_HEADER_BYTES, reinterpret_cast<cudaStream_t>(stream)) !=
-      cudaSuccess)
-    return QSA_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, QSA_WS_HEADER_BYTES, s) != cudaSuccess) return QSA_ERR_CUDA;
   return qsa_decode(q, cache, q_idx, w, out, h_len, sel_idx, sel_cnt, ws,
                     QSA_NOALLOC_SCRATCH_BYTES, params, stream);
+}
+
+extern "C" qsa_status qsa_noalloc_last_device_error(qsa_stream_t stream, uint32_t* site) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t h[4] = {0, 0, 0, 0};
+  if (cudaMemcpyFromSymbolAsync(h, g_noalloc_scratch, sizeof(h), 0, cudaMemcpyDeviceToHost, s) !=
+      cudaSuccess)
+    return QSA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return QSA_ERR_CUDA;
+  if (h[0] != 0) {
+    static const uint32_t zero[4] = {0, 0, 0, 0};
+    if (cudaMemcpyToSymbolAsync(g_noalloc_scratch, zero, sizeof(zero), 0, cudaMemcpyHostToDevice,
+                                s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+      return QSA_ERR_CUDA;
+  }
+  if (site) *site = h[1];
+  if (h[0] == 0) return QSA_OK;
+  return h[0] == kErrTimeout ? QSA_ERR_TIMEOUT : QSA_ERR_DEVICE;
 }

@@ -97,7 +97,11 @@ struct AttnArgs {
   float* part_m;           // decode: [B][2][splits][12]
   float* part_l;
   DevStatus st;
+  int32_t fault_tile = -1; // testing only (-1: off): see k_sparse_attn
 };
+
+// Testing only: the wait limit of the faulted tile's MMA warp (1 ms).
+constexpr uint64_t kFaultWaitNs = 1000000ull;
 
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   return (static_cast<uint64_t>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
@@ -125,7 +129,9 @@ __device__ __forceinline__ float ex2_approx(float x) {
 // (and the run of padding slots past the end of the union) are cut into power-of-two pieces;
 // the first lane of each run issues one TMA box per piece (rows 4*blk.., two 64-dim panels).
 // Run r of a chunk (in slot order) goes to warp r mod nw; warp 0 posts the chunk's bytes.
-// Padding rows come from an out-of-range coordinate and are zero-filled.  kPaged (a paged
+// Padding rows come from an out-of-range coordinate and are zero-filled.  skip_first (testing
+// only): nothing is posted or copied for the first chunk, so its full barrier never completes
+// and the consumer's bounded wait gives up; that chunk is then not drained.  kPaged (a paged
 // decode cache): runs are also cut where a page starts, and each run's rows are looked up in
 // the page table of sequence seq (KV head g).  The other instances carry none of that code: the
 // prefill gather is limited by how fast these warps issue copies.
@@ -136,7 +142,7 @@ __device__ __forceinline__ void attn_producer(const CUtensorMap* maps, unsigned 
                                               int64_t kv_row_base, int col0, int32_t oob_row,
                                               const Paging& pg, int seq, int g,
                                               int w, int nw, volatile int* abort, DevStatus st,
-                                              uint32_t site) {
+                                              uint32_t site, bool skip_first) {
   const int lane = threadIdx.x & 31;
   int upos = c_begin * AttnCfg::kChunkBlocks + lane;
   int blk_next = upos < U ? uni[upos] : -1;
@@ -161,7 +167,8 @@ __device__ __forceinline__ void attn_producer(const CUtensorMap* maps, unsigned 
     if (lane == 0) ok = mbar_wait(&empty[s], ((i / stages) & 1) ^ 1, abort, st, site);
     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
     if (!ok) break;
-    if (lane == 0 && w == 0) mbar_arrive_expect_tx(&full[s], AttnCfg::kKVBytes);
+    const bool skip = skip_first && i == 0;
+    if (lane == 0 && w == 0 && !skip) mbar_arrive_expect_tx(&full[s], AttnCfg::kKVBytes);
     __syncwarp();
     const int prev = __shfl_up_sync(0xffffffffu, blk, 1);
     bool start = lane == 0 || (blk < 0) != (prev < 0) || (blk >= 0 && blk != prev + 1);
@@ -169,7 +176,7 @@ __device__ __forceinline__ void attn_producer(const CUtensorMap* maps, unsigned 
     const unsigned starts = __ballot_sync(0xffffffffu, start);
     // (a box may complete before warp 0 posts the bytes: the phase cannot end while the
     // posting arrival is missing)
-    if (start && __popc(starts & ((1u << lane) - 1u)) % nw == w) {
+    if (!skip && start && __popc(starts & ((1u << lane) - 1u)) % nw == w) {
       const unsigned later = starts & ~((2u << lane) - 1u);   // run starts after this lane
       const int run_end = later ? __ffs(later) - 1 : 32;
       int off = 0;
@@ -200,7 +207,8 @@ __device__ __forceinline__ void attn_producer(const CUtensorMap* maps, unsigned 
     ++issued;
   }
   if (lane == 0 && *abort) {
-    const int from = issued > stages ? issued - stages : 0;
+    int from = issued > stages ? issued - stages : 0;
+    if (skip_first && from == 0) from = 1;   // nothing was posted for the skipped chunk
     for (int j = from; j < issued; ++j) mbar_drain(&full[j % stages], (j / stages) & 1);
   }
 }
@@ -270,6 +278,10 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // Testing only (args.fault_tile >= 0): in that tile (KV head 0, first split) the K producers
+  // post nothing for the first chunk and the MMA warp's waits give up after kFaultWaitNs, so
+  // the launch reports QSA_ERR_TIMEOUT (site 23) and every warp unwinds through the abort path.
+  const bool fault = args.fault_tile >= 0 && tile == args.fault_tile && g == 0 && split == 0;
 
   if (nchunks == 0 || ntok == 0) {
     // decode split without keys: write an empty partial
@@ -355,7 +367,7 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
     __syncwarp();
     attn_producer<kPaged>(maps.k, sK, k_full, k_empty, C::kKStages, uni, U, c_begin, nchunks,
                   kv_row_base, col0, args.oob_row, args.pg, tile, g, kw, C::kKWarps, s_abort,
-                  args.st, 20);
+                  args.st, 20, fault);
     if (kw == 0 && lane == 0 && *s_abort) mbar_drain(q_full, 0);
   } else if (warp >= C::kVWarp0) {
     // ---------------- V producers ----------------
@@ -365,17 +377,18 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
     __syncwarp();
     attn_producer<kPaged>(maps.v, sV, v_full, v_empty, C::kVStages, uni, U, c_begin, nchunks,
                   kv_row_base, col0, args.oob_row, args.pg, tile, g, vw, C::kVWarps, s_abort,
-                  args.st, 27);
+                  args.st, 27, false);
   } else {
     // ---------------- MMA issuer (warp kMmaWarp) ----------------
     if (lane == 0) {
       const uint32_t sQ0 = smem_u32(sQ);
-      bool ok = mbar_wait(q_full, 0, s_abort, args.st, 21);
+      const uint64_t lim = fault ? kFaultWaitNs : kWaitLimitNs;
+      bool ok = mbar_wait(q_full, 0, s_abort, args.st, 21, lim);
       auto issue_pv = [&](int j) -> bool {
         const int bj = j & 1;
         const int vs = j % C::kVStages;
-        if (!mbar_wait(&p_full[bj], (j >> 1) & 1, s_abort, args.st, 22)) return false;
-        if (!mbar_wait(&v_full[vs], (j / C::kVStages) & 1, s_abort, args.st, 28)) return false;
+        if (!mbar_wait(&p_full[bj], (j >> 1) & 1, s_abort, args.st, 22, lim)) return false;
+        if (!mbar_wait(&v_full[vs], (j / C::kVStages) & 1, s_abort, args.st, 28, lim)) return false;
         tc_fence_after();
         const uint32_t sV0 = smem_u32(sV + vs * C::kKVBytes);
 #pragma unroll
@@ -393,12 +406,12 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
       for (int i = 0; ok && i < nchunks; ++i) {
         const int b = i & 1;
         const int ks = i % C::kKStages;
-        if (!mbar_wait(&k_full[ks], (i / C::kKStages) & 1, s_abort, args.st, 23)) break;
+        if (!mbar_wait(&k_full[ks], (i / C::kKStages) & 1, s_abort, args.st, 23, lim)) break;
         // S_i overwrites the TMEM buffer that held P_{i-2}: P_{i-2}.V must have completed
         // (tcgen05 MMAs in flight are not ordered against each other's TMEM accesses).  In
         // decode P has its own buffer, which the softmax rewrites only after S_i is in, so
         // the same wait orders that rewrite after P_{i-2}.V.
-        if (i >= 2 && !mbar_wait(&p_free[b], ((i - 2) >> 1) & 1, s_abort, args.st, 29)) break;
+        if (i >= 2 && !mbar_wait(&p_free[b], ((i - 2) >> 1) & 1, s_abort, args.st, 29, lim)) break;
         tc_fence_after();
         const uint32_t sK0 = smem_u32(sK + ks * C::kKVBytes);
 #pragma unroll

@@ -130,7 +130,15 @@ __device__ __forceinline__ ScoreWork<NTOK> score_work(const ScoreArgs& a) {
     const int b = static_cast<int>(blockIdx.x) / a.splits;
     const int split = static_cast<int>(blockIdx.x) % a.splits;
     const int p = a.len[b] - 1;
-    const int n_c = p >= 0 ? p / kBlock : 0;
+    int n_c = p >= 0 ? p / kBlock : 0;
+    // The grid covers the blocks of the host lengths the caller passed.  A device length
+    // beyond them (a stale host copy) is reported, and only the covered blocks are scored;
+    // the top-k then sees that same count, so it never reads a score that was not written.
+    const int covered = a.splits * a.mtiles_per_split * 128;
+    if (n_c > covered) {
+      if (split == 0 && threadIdx.x == 0) report_error(a.st, kErrDevice, 207);
+      n_c = covered;
+    }
     if (split == 0 && threadIdx.x == 0 && a.n_c_out) a.n_c_out[b] = n_c;
     const int total = (n_c + 127) / 128;
     const int m0 = split * a.mtiles_per_split;

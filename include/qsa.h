@@ -26,6 +26,9 @@
  *   - All tensor arguments are DEVICE pointers, 16-byte aligned, contiguous, row-major in
  *     the layouts stated, owned by the caller.  The library never allocates device memory;
  *     scratch space is the caller's `workspace` (size from the *_workspace_size query).
+ *     The one exception is qsa_decode_noalloc below: its scratch is a static device array
+ *     of QSA_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads the
+ *     library holds until the process exits.
  *   - `h_*` arguments are HOST pointers read synchronously during the call.
  *   - Work is enqueued on `stream` (NULL = the legacy default stream) and the call returns
  *     without synchronising.  Host-detectable errors are returned before anything is
@@ -33,8 +36,9 @@
  *     range) are recorded in the first 16 bytes of the workspace and reported by
  *     qsa_last_device_error().
  *   - bf16 means IEEE bfloat16 (raw 16-bit); fp32 is IEEE single.
- *   - Calls are re-entrant; the only global state is a per-device cache of driver entry
- *     points.  Concurrent calls must not share a workspace.
+ *   - Calls are re-entrant; the only global state is the cached driver entry point for
+ *     tensor-map encoding, and, for qsa_decode_noalloc, its static scratch array and the
+ *     per-device address of that array.  Concurrent calls must not share a workspace.
  */
 #ifndef QSA_H_
 #define QSA_H_
@@ -85,6 +89,13 @@ typedef struct {
                               0 = library default (one wave of CTAs: SMs / (2 x batch)) */
   int32_t score_chunk_rows;/* prefill: query rows scored per pass (bounds the score
                               buffer in the workspace); 0 = library default */
+  int32_t debug_fault;     /* testing only; 0 in normal use.  1: in the prefill attention the
+                              last tile's KV head 0 posts nothing for its first key chunk and
+                              that tile's MMA waits give up after 1 ms, so the call's device
+                              status reads QSA_ERR_TIMEOUT (site 23) and that tile's output is
+                              undefined.  It exercises the bounded-wait unwind (copies in
+                              flight drained, tensor memory freed): a normal call may follow at
+                              once.  Other values are refused (QSA_ERR_INVALID_ARG). */
 } qsa_params;
 
 /* KV cache for decode.  Blocks of 4 tokens are contiguous per (sequence, KV head):
@@ -238,19 +249,27 @@ QSA_API qsa_status qsa_decode(const void *q, const qsa_cache *cache, const void 
  *     and budget need more scratch than that (compare qsa_decode_workspace_size); batch 64 at
  *     capacity 262,144 with budget 512 needs about 19 MB.
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
- *   - The first call on a device looks up the array's device address with that device
- *     current; make that first call before any stream capture.
+ *   - Every call made outside a stream capture looks up the array's device address on the
+ *     current device (so a module reloaded after cudaDeviceReset is followed).  A call made
+ *     during a capture reuses the address of the last uncaptured call on that device: make
+ *     one call before any stream capture, or the captured call fails with QSA_ERR_CUDA.
  *   - Every call, on every stream, shares the one array and it keeps the last call's
  *     contents; each call clears the status words at its start.  Calls that overlap on the
  *     GPU race on the array and corrupt each other's results: serialise them (one stream,
- *     or events between streams).  Device-side status words of these calls cannot be read
- *     back by the caller. */
+ *     or events between streams).  Read a call's device-side status with
+ *     qsa_noalloc_last_device_error before the next call clears it. */
 #define QSA_NOALLOC_SCRATCH_BYTES (32u << 20)
 
 QSA_API qsa_status qsa_decode_noalloc(const void *q, const qsa_cache *cache, const void *q_idx,
                                       const void *w, void *out, const int32_t *h_len,
                                       int32_t *sel_idx, int32_t *sel_cnt, qsa_params params,
                                       qsa_stream_t stream);
+
+/* The device-side status of the last qsa_decode_noalloc call, read from the library's static
+ * scratch array: synchronises `stream`, then returns and clears it exactly as
+ * qsa_last_device_error does for a workspace (QSA_OK, QSA_ERR_TIMEOUT, QSA_ERR_DEVICE, or
+ * QSA_ERR_CUDA when the copy or the synchronisation failed).  Allocates nothing. */
+QSA_API qsa_status qsa_noalloc_last_device_error(qsa_stream_t stream, uint32_t *site);
 
 /* ---------------------------------------------------------------------------------- */
 /* Paged KV cache (aiany.app "Qwen3.8-Flash-Next", "Implementation notes": the model ships

@@ -88,6 +88,12 @@ def test_host_side_argument_errors():
     r = lib.qsa_prefill(_p(good), _p(good), _p(good), _p(good), _p(good), _p(good), _p(good), cu, 1,
                         _p(good), _p(good), 1 << 30, B._params(0), None)
     assert B.STATUS[r] == "QSA_ERR_INVALID_ARG"
+    # the testing fault hook takes 0 or 1 only, and is prefill-only
+    r = lib.qsa_prefill(_p(good), _p(good), _p(good), _p(good), _p(good), _p(good), _p(good), cu, 1,
+                        _p(good), _p(good), 1 << 30, B._params(16, debug_fault=2), None)
+    assert B.STATUS[r] == "QSA_ERR_INVALID_ARG"
+    desc = B.CacheDesc(good, good, good, good, good, 2, 64)
+    assert lib.qsa_decode_workspace_size(ctypes.byref(desc), B._params(16, debug_fault=1)) == 0
     # append beyond capacity
     desc = B.CacheDesc(good, good, good, good, good, 2, 64)
     h_len = (ctypes.c_int32 * 2)(60, 10)

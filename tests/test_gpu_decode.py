@@ -33,10 +33,11 @@ def _oracle_row(k_tok, v_tok, kidx_tok, q, q_idx, w, topk, forced=None):
 
 
 def _decode_session(spec, check_seqs, steps, splits=0, device_gen=False, ctx_fn=None,
-                    step_fn=None, exact_sel=False, cache_fn=None):
+                    step_fn=None, exact_sel=False, cache_fn=None, check_steps=None):
     """ctx_fn(k, v, k_idx) and step_fn(step dict) may reshape the seeded inputs (ties);
     exact_sel demands the oracle's selection itself (inputs whose scores are exact);
-    cache_fn(spec) builds the cache (default: a contiguous KVCache)."""
+    cache_fn(spec) builds the cache (default: a contiguous KVCache); check_steps lists the
+    steps compared with the oracle (default: every step)."""
     gen_dev = DEV if device_gen else "cpu"
     k_ctx, v_ctx, ki_ctx = W.decode_context(spec, device=gen_dev)
     if ctx_fn is not None:
@@ -56,6 +57,7 @@ def _decode_session(spec, check_seqs, steps, splits=0, device_gen=False, ctx_fn=
     seqs = {b: (k_ctx[b, :spec.context[b]].cpu(), v_ctx[b, :spec.context[b]].cpu(),
                 ki_ctx[b, :spec.context[b]].cpu()) for b in check_seqs}
     del k_ctx, v_ctx, ki_ctx
+    added = {b: ([], [], []) for b in check_seqs}   # tokens appended since the last check
     results = []
     for step in range(steps):
         st = W.decode_step(spec, step, device=gen_dev)
@@ -67,11 +69,17 @@ def _decode_session(spec, check_seqs, steps, splits=0, device_gen=False, ctx_fn=
         torch.cuda.synchronize()
         assert dec.device_error() == ("QSA_OK", 0)
         for b in check_seqs:
+            for lst, key in zip(added[b], ("k", "v", "k_idx")):
+                lst.append(st[key][b].cpu())
+        if check_steps is not None and step not in check_steps:
+            continue
+        for b in check_seqs:
             kt, vt, kit = seqs[b]
-            kt = torch.cat([kt, st["k"][b].cpu()])
-            vt = torch.cat([vt, st["v"][b].cpu()])
-            kit = torch.cat([kit, st["k_idx"][b].cpu()])
+            kt = torch.cat([kt] + added[b][0])
+            vt = torch.cat([vt] + added[b][1])
+            kit = torch.cat([kit] + added[b][2])
             seqs[b] = (kt, vt, kit)
+            added[b] = ([], [], [])
             q, qi, w = st["q"][b].cpu(), st["q_idx"][b].cpu(), st["w"][b].cpu()
             o_idx, o_cnt, o_kth, _, kbar = _oracle_row(kt, vt, kit, q, qi, w, spec.topk)
             g_idx = idx[b:b + 1].cpu().numpy()
@@ -166,8 +174,15 @@ def test_decode_256k_four_sequences():
 
 @pytest.mark.slow
 def test_decode_1m_incremental():
+    # the extended-context case as specified: 4 sequences at 1,048,509..1,048,512 tokens,
+    # 64 consecutive append + decode steps, so that 16 blocks per sequence complete by
+    # incremental compression; the oracle checks the first and the last step of every
+    # sequence, including the compressed cache bit for bit after the last append
     spec = W.decode_spec("decode1m")
-    _decode_session(spec, check_seqs=[0, 3], steps=4, device_gen=True)
+    assert spec.steps == 64
+    res = _decode_session(spec, check_seqs=[0, 1, 2, 3], steps=spec.steps, device_gen=True,
+                          check_steps={0, spec.steps - 1})
+    assert len(res) == 8
 
 
 def test_decode_batch_of_40_mixed_contexts():
