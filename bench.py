@@ -392,6 +392,152 @@ def run_qsa(args, rank, world, local):
 
 
 # ------------------------------------------------------------------------------------
+def ragged_attention_flops(lengths, k=TOPK):
+    return sum(prefill_attention_flops(L, k) for L in lengths)
+
+
+def ragged_indexer_flops(lengths):
+    return sum(prefill_indexer_flops(L) for L in lengths)
+
+
+def run_mixed(args, rank, world, local):
+    """The mixed ragged workload, timed after the headline parts, each on its own:
+    * a varlen prefill of 8 sequences of 1,000..131,071 tokens (not multiples of 4);
+    * decode of 4 sequences at 1,048,509..1,048,512 tokens of context, 64 consecutive
+      append + decode steps captured as one CUDA graph (so 16 blocks per sequence are
+      completed by incremental compression inside every replay)."""
+    import torch
+    import block_sparse_attention_40_b200 as qsa
+    from block_sparse_attention_40_b200 import binding as B
+    from block_sparse_attention_40_b200 import workloads as W
+
+    dev = torch.device(f"cuda:{local}")
+    stream = torch.cuda.current_stream(dev)
+    peaks, peak_src = load_peaks()
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_rd = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+
+    def flush():
+        flush_buf.random_(0, 255)
+        flush_rd.sum()
+
+    out = {}
+    K = args.steps
+    clocks = ClockSampler(local)
+    clocks.start()
+    launches0 = B.launch_count()
+    graph_launches = 0
+    # ---- varlen prefill ----
+    p = W.prefill("ragged", device=dev, seed=1004 + rank)
+    lens = (p.cu_seqlens[1:] - p.cu_seqlens[:-1]).tolist()
+    T = p.total_tokens
+    ctx = qsa.Prefill(p.cu_seqlens, dev, TOPK)
+    idx = torch.empty((T, TOPK), dtype=torch.int32, device=dev)
+    cnt = torch.empty((T,), dtype=torch.int32, device=dev)
+    o = torch.empty_like(p.q)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    for i in range(args.warmup + K):
+        flush()
+        e = ev[i - args.warmup] if i >= args.warmup else None
+        if e:
+            e[0].record(stream)
+        ctx.select(p.q_idx, p.k_idx, p.w, idx, cnt)
+        if e:
+            e[1].record(stream)
+        ctx.attend(p.q, p.k, p.v, idx, cnt, o)
+        if e:
+            e[2].record(stream)
+    torch.cuda.synchronize(dev)
+    assert ctx.device_error() == ("QSA_OK", 0)
+    sel = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev) / K, world, dev)
+    att = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in ev) / K, world, dev)
+    af, xf = ragged_attention_flops(lens), ragged_indexer_flops(lens)
+    out["prefill_ragged"] = {
+        "lengths": lens, "tokens": T, "ms": sel + att, "select_ms": sel, "attention_ms": att,
+        "tokens_per_s": world * T / ((sel + att) / 1e3),
+        "roofline": {"kernel": "qsa_sparse_attention", "bound": "tensor",
+                     "achieved": af / (att / 1e3) / 1e12, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": af / (att / 1e3) / 1e12 / peaks["bf16_tflops"],
+                     "peak_source": f"{peak_src} bf16 burst",
+                     "algorithmic": f"{af / 1e12:.4f} TFLOP selected-token per launch"},
+        "indexer_tflop": xf / 1e12}
+    del p, ctx, idx, cnt, o
+    torch.cuda.empty_cache()
+    # ---- 1M decode, 64 append + decode steps per replay ----
+    spec = W.decode_spec("decode1m")
+    spec.seed += 17 * rank
+    cache = qsa.KVCache(spec.batch, spec.capacity, dev, zero=False)
+    kc, vc, kic = W.decode_context(spec, device=dev)
+    lmax = max(spec.context)
+    for c0 in range(0, lmax, 16384):
+        c1 = min(lmax, c0 + 16384)
+        counts = [max(0, min(c1, L) - c0) for L in spec.context]
+        cache.append(kc[:, c0:c1].contiguous(), vc[:, c0:c1].contiguous(),
+                     kic[:, c0:c1].contiguous(), counts=counts)
+    del kc, vc, kic
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
+    saved = (cache.len.clone(), cache.kbar_partial.clone(), list(cache.h_len))
+    dec = qsa.Decoder(cache, TOPK)
+    steps = [W.decode_step(spec, s, device=dev) for s in range(spec.steps)]
+    outs = torch.empty((spec.steps, spec.batch, 24, 128), dtype=torch.bfloat16, device=dev)
+
+    def reset():
+        cache.len.copy_(saved[0])
+        cache.kbar_partial.copy_(saved[1])
+        cache.h_len = list(saved[2])
+
+    def run_steps():
+        for s, st in enumerate(steps):
+            cache.append(st["k"], st["v"], st["k_idx"])
+            dec.run(st["q"], st["q_idx"], st["w"], out=outs[s])
+
+    for _ in range(args.warmup):
+        reset()
+        run_steps()
+    reset()
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    n0 = B.launch_count()
+    with torch.cuda.graph(g):
+        run_steps()
+    torch.cuda.synchronize(dev)
+    per_replay = B.launch_count() - n0
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    for i in range(args.warmup + K):
+        reset()
+        flush()
+        e = ev[i - args.warmup] if i >= args.warmup else None
+        if e:
+            e[0].record(stream)
+        g.replay()
+        if e:
+            e[1].record(stream)
+    torch.cuda.synchronize(dev)
+    assert dec.device_error() == ("QSA_OK", 0)
+    graph_launches = per_replay * (args.warmup + K)
+    ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev) / K, world, dev)
+    nbytes = sum(decode_bytes_per_seq(L + s + 1) for L in spec.context for s in range(spec.steps))
+    gbs = nbytes / (ms / 1e3) / 1e9
+    out["decode_1m"] = {
+        "batch": spec.batch, "context": spec.context, "steps_per_replay": spec.steps,
+        "ms_per_replay": ms, "ms_per_step": ms / spec.steps,
+        "tokens_per_s": world * spec.batch * spec.steps / (ms / 1e3),
+        "timing": "cuda graph of 64 x (append 1 token + decode), replayed; cache lengths reset "
+                  "between replays; L2 flushed before each replay",
+        "roofline": {"kernel": "64 whole decode steps", "bound": "hbm", "achieved": gbs,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                     "peak_source": f"{peak_src} HBM copy",
+                     "algorithmic": f"{nbytes / spec.steps / spec.batch / 1e6:.2f} MB per "
+                                    f"sequence per step"}}
+    g.reset()
+    out["clocks"] = clocks.stop()
+    # kernels this part launched, warm-ups included (graph replays count their kernels; the
+    # capture itself launches nothing)
+    out["gpu_launches_incl_warmup"] = B.launch_count() - launches0 + graph_launches - per_replay
+    return out
+
+
 def cpu_baseline(seconds_target=12.0, threads=None):
     """The oracle, as it stands, on a bounded sample of the 64K prefill rows."""
     import numpy as np
@@ -459,6 +605,9 @@ def main():
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="time the decode step as eager launches instead of a CUDA graph replay")
     ap.add_argument("--no-cpu-baseline", dest="cpu", action="store_false")
+    ap.add_argument("--no-mixed", dest="mixed", action="store_false",
+                    help="skip the mixed ragged workload (8-sequence varlen prefill and the "
+                         "1M-context decode) that follows the headline parts")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -467,6 +616,11 @@ def main():
         run_reference(args, rank, world)
         return
     r = run_qsa(args, rank, world, local)
+    mixed = None
+    if args.mixed and args.workload == "both":
+        import torch
+        torch.cuda.empty_cache()
+        mixed = run_mixed(args, rank, world, local)
     if rank != 0:
         return
     K = args.steps
@@ -531,6 +685,9 @@ def main():
         line["e2e"] = r["e2e"]["prefill"]
     elif "decode" in r["e2e"]:
         line["e2e"] = r["e2e"]["decode"]
+    if mixed is not None:
+        # the mixed ragged workload, timed separately after the headline step
+        line["mixed_ragged"] = mixed
     if args.cpu and world == 1:
         line["cpu_baseline"] = cpu_baseline()
     print(json.dumps(line), flush=True)

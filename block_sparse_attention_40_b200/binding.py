@@ -31,7 +31,9 @@ EXPORTS = ("qsa_status_string", "qsa_version", "qsa_launch_count", "qsa_workspac
            "qsa_prefill_workspace_size", "qsa_prefill", "qsa_prefill_select",
            "qsa_sparse_attention", "qsa_append_kv", "qsa_decode_workspace_size", "qsa_decode",
            "qsa_decode_noalloc", "qsa_noalloc_last_device_error", "qsa_append_kv_paged",
-           "qsa_decode_paged_workspace_size", "qsa_decode_paged")
+           "qsa_decode_paged_workspace_size", "qsa_decode_paged",
+           "qsa_decode_shard_workspace_size", "qsa_decode_shard_select", "qsa_merge_candidates",
+           "qsa_decode_shard_attend", "qsa_combine_partials")
 
 
 class QSAError(RuntimeError):
@@ -97,6 +99,11 @@ def load(build_if_needed: bool = True):
             "qsa_append_kv_paged": ([P, P, P, P, I32, P, P, P], st),
             "qsa_decode_paged_workspace_size": ([P, Params], SZ),
             "qsa_decode_paged": ([P, P, P, P, P, P, P, P, P, SZ, Params, P], st),
+            "qsa_decode_shard_workspace_size": ([P, Params], SZ),
+            "qsa_decode_shard_select": ([P, P, P, I32, P, P, P, P, P, P, SZ, Params, P], st),
+            "qsa_merge_candidates": ([P, P, P, I32, I32, I32, I32, P, P, P, SZ, P], st),
+            "qsa_decode_shard_attend": ([P, P, I32, P, P, P, P, P, P, P, SZ, Params, P], st),
+            "qsa_combine_partials": ([P, P, P, I32, I32, P, P], st),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -506,3 +513,94 @@ def noalloc_device_error(device) -> tuple:
     site = ctypes.c_uint32(0)
     code = load().qsa_noalloc_last_device_error(_stream(torch.device(device)), ctypes.byref(site))
     return STATUS.get(code, str(code)), int(site.value)
+
+
+# --------------------------------------------------------------------------------------
+class ShardDecoder:
+    """Decode over one shard of a context split across caches (see include/qsa.h, context-
+    sharded decode): the shard holds tokens [4 * block0, 4 * block0 + capacity) of every
+    sequence of the batch, block0 a multiple of 128."""
+
+    def __init__(self, cache: KVCache, block0: int, topk=512):
+        if isinstance(cache, PagedKVCache):
+            raise TypeError("a shard is a contiguous cache")
+        self.cache, self.block0, self.topk = cache, int(block0), int(topk)
+        self.params = _params(topk)
+        self.lib = load()
+        desc = cache.desc()
+        n = self.lib.qsa_decode_shard_workspace_size(ctypes.byref(desc), self.params)
+        if n == 0:
+            raise QSAError("qsa_decode_shard_workspace_size", 1)
+        self.ws = new_workspace(n, cache.device)
+
+    def select(self, q_idx, w, glen: torch.Tensor, cand_score=None, cand_idx=None,
+               cand_cnt=None):
+        """This shard's candidates: (scores [B, topk] fp32, global blocks [B, topk] int32,
+        counts [B] int32).  glen: the sequences' whole lengths, int32 [B] on the device."""
+        B = self.cache.batch
+        _need(q_idx, "q_idx", torch.bfloat16, (IDX_HEADS, IDX_DIM), 3)
+        _need(w, "w", torch.bfloat16, (IDX_HEADS,), 2)
+        _need(glen, "glen", torch.int32, ndim=1)
+        dev = self.cache.device
+        if cand_score is None:
+            cand_score = torch.empty((B, self.topk), dtype=torch.float32, device=dev)
+            cand_idx = torch.empty((B, self.topk), dtype=torch.int32, device=dev)
+            cand_cnt = torch.empty((B,), dtype=torch.int32, device=dev)
+        h_len = (ctypes.c_int32 * B)(*self.cache.h_len)
+        desc = self.cache.desc()
+        _check("qsa_decode_shard_select", self.lib.qsa_decode_shard_select(
+            _ptr(q_idx), _ptr(w), ctypes.byref(desc), self.block0, _ptr(glen), h_len,
+            _ptr(cand_score), _ptr(cand_idx), _ptr(cand_cnt), _ptr(self.ws), self.ws.numel(),
+            self.params, _stream(dev)))
+        return cand_score, cand_idx, cand_cnt
+
+    def attend(self, q, glen, sel_idx, sel_cnt, part_o=None, part_m=None, part_l=None):
+        """This shard's partial softmax: (o [B, 24, 128], m [B, 24], l [B, 24]) fp32."""
+        B = self.cache.batch
+        _need(q, "q", torch.bfloat16, (NUM_HEADS, HEAD_DIM), 3)
+        dev = self.cache.device
+        if part_o is None:
+            part_o = torch.empty((B, NUM_HEADS, HEAD_DIM), dtype=torch.float32, device=dev)
+            part_m = torch.empty((B, NUM_HEADS), dtype=torch.float32, device=dev)
+            part_l = torch.empty((B, NUM_HEADS), dtype=torch.float32, device=dev)
+        desc = self.cache.desc()
+        _check("qsa_decode_shard_attend", self.lib.qsa_decode_shard_attend(
+            _ptr(q), ctypes.byref(desc), self.block0, _ptr(glen), _ptr(sel_idx), _ptr(sel_cnt),
+            _ptr(part_o), _ptr(part_m), _ptr(part_l), _ptr(self.ws), self.ws.numel(),
+            self.params, _stream(dev)))
+        return part_o, part_m, part_l
+
+    def device_error(self):
+        return last_device_error(self.ws)
+
+
+def merge_candidates(cand_score, cand_idx, cand_cnt, topk: int, max_blocks: int, sel_idx=None,
+                     sel_cnt=None, workspace=None):
+    """Stacked shard candidates [R, B, topk] (scores, blocks) and counts [R, B] -> the
+    selection (idx [B, topk] ascending -1 padded, cnt [B])."""
+    _need(cand_score, "cand_score", torch.float32, ndim=3)
+    _need(cand_idx, "cand_idx", torch.int32, ndim=3)
+    _need(cand_cnt, "cand_cnt", torch.int32, ndim=2)
+    R, B, k = cand_score.shape
+    dev = cand_score.device
+    if sel_idx is None:
+        sel_idx = torch.empty((B, topk), dtype=torch.int32, device=dev)
+        sel_cnt = torch.empty((B,), dtype=torch.int32, device=dev)
+    ws = workspace if workspace is not None else new_workspace(WS_HEADER_BYTES, dev)
+    _check("qsa_merge_candidates", load().qsa_merge_candidates(
+        _ptr(cand_score), _ptr(cand_idx), _ptr(cand_cnt), R, B, int(topk), int(max_blocks),
+        _ptr(sel_idx), _ptr(sel_cnt), _ptr(ws), ws.numel(), _stream(dev)))
+    return sel_idx, sel_cnt
+
+
+def combine_partials(part_o, part_m, part_l, out=None):
+    """Stacked shard partials o [R, B, 24, 128], m and l [R, B, 24] -> out [B, 24, 128] bf16."""
+    _need(part_o, "part_o", torch.float32, (NUM_HEADS, HEAD_DIM), 4)
+    _need(part_m, "part_m", torch.float32, (NUM_HEADS,), 3)
+    _need(part_l, "part_l", torch.float32, (NUM_HEADS,), 3)
+    R, B = part_o.shape[:2]
+    if out is None:
+        out = torch.empty((B, NUM_HEADS, HEAD_DIM), dtype=torch.bfloat16, device=part_o.device)
+    _check("qsa_combine_partials", load().qsa_combine_partials(
+        _ptr(part_o), _ptr(part_m), _ptr(part_l), R, B, _ptr(out), _stream(part_o.device)))
+    return out

@@ -779,14 +779,73 @@ size_t qsa_decode_paged_workspace_size(const qsa_paged_cache* cache, qsa_params 
 }  // extern "C"
 
 namespace {
+// Decode attention (a6) over the one-token plan records in `plan`: the output directly (one
+// split, partials false) or the split partials (m, l, o).
+qsa_status launch_decode_attention(const void* q, const CacheView& view, const DecodeGeom& g,
+                                   const int32_t* plan, DevStatus dst, void* out, int splits,
+                                   float* part_o, float* part_m, float* part_l, bool partials,
+                                   cudaStream_t s) {
+  const qsa_cache* cache = view.c;
+  AttnMaps maps;
+  const uint64_t dq[3] = {128, 24, static_cast<uint64_t>(g.B)};
+  const uint64_t sq[2] = {256, 24 * 256};
+  const uint32_t bq[3] = {64, 12, 1};
+  if (!make_tmap(&maps.q, q, 3, dq, sq, bq)) return QSA_ERR_CUDA;
+  const uint64_t dkv[2] = {128, static_cast<uint64_t>(view.kv_rows)};
+  const uint64_t skv[1] = {256};
+  for (int j = 0; j < kNumBoxSizes; ++j) {
+    const uint32_t bkv[2] = {64, 4u << j};
+    if (!make_tmap(&maps.k[j], cache->k_blocks, 2, dkv, skv, bkv)) return QSA_ERR_CUDA;
+    if (!make_tmap(&maps.v[j], cache->v_blocks, 2, dkv, skv, bkv)) return QSA_ERR_CUDA;
+  }
+  const qsa_status pst = prepare_attention();
+  if (pst != QSA_OK) return pst;
+  if (view.kv_rows >= 0x7fffffffll) return QSA_ERR_UNSUPPORTED;
+  AttnArgs a{};
+  a.oob_row = static_cast<int32_t>(view.kv_rows);
+  a.pg = view.pg;
+  a.plan = plan;
+  a.pl = g.pl;
+  a.decode = 1;
+  a.splits = splits;
+  a.cap_blocks = g.cap / 4;
+  a.part_o = part_o;
+  a.part_m = part_m;
+  a.part_l = part_l;
+  a.st = dst;
+  a.fault_tile = -1;
+  a.partials = partials ? 1 : 0;
+  a.out = reinterpret_cast<__nv_bfloat16*>(out);   // written directly with one split
+  dim3 grid(g.B, 2, splits);
+  if (view.pg.table != nullptr) {
+    QSA_CHECK_PDL(launch_pdl(k_sparse_attn<true, true>, grid, dim3(AttnCfg::kThreads),
+                             AttnCfg::kSmemBytes, s, maps, a));
+  } else {
+    QSA_CHECK_PDL(launch_pdl(k_sparse_attn<true>, grid, dim3(AttnCfg::kThreads),
+                             AttnCfg::kSmemBytes, s, maps, a));
+  }
+  return QSA_OK;
+}
+
+// One shard of a context split over several caches (context-sharded decode).
+struct ShardOpt {
+  const int32_t* glen = nullptr;   // device [B]: the sequences' whole lengths
+  int32_t block0 = 0;              // global block of the shard's first block
+  float* cand_score = nullptr;     // selection only: scores of the proposed blocks
+};
+
 qsa_status decode_impl(const void* q, const CacheView& view, const void* q_idx, const void* w,
                        void* out, const int32_t* h_len, int32_t* sel_idx, int32_t* sel_cnt,
-                       void* workspace, size_t ws_bytes, qsa_params params, qsa_stream_t stream) {
+                       void* workspace, size_t ws_bytes, qsa_params params, qsa_stream_t stream,
+                       const ShardOpt* shard = nullptr) {
   const qsa_cache* cache = view.c;
   if (!cache || !h_len) return QSA_ERR_INVALID_ARG;
-  qsa_status st = check_prefill_ptrs({q, q_idx, w, out, workspace, cache->k_blocks,
-                                      cache->v_blocks, cache->kbar, cache->len});
+  qsa_status st = shard ? check_prefill_ptrs({q_idx, w, workspace, cache->kbar, cache->len,
+                                              shard->glen, shard->cand_score, sel_idx, sel_cnt})
+                        : check_prefill_ptrs({q, q_idx, w, out, workspace, cache->k_blocks,
+                                              cache->v_blocks, cache->kbar, cache->len});
   if (st != QSA_OK) return st;
+  if (shard && (shard->block0 < 0 || shard->block0 % 128 != 0)) return QSA_ERR_INVALID_ARG;
   if ((sel_idx && !aligned16(sel_idx)) || (sel_cnt && !aligned16(sel_cnt))) return QSA_ERR_ALIGNMENT;
   DecodeGeom g;
   st = decode_geom(cache, params, &g);
@@ -794,7 +853,7 @@ qsa_status decode_impl(const void* q, const CacheView& view, const void* q_idx, 
   if (ws_bytes < g.total) return QSA_ERR_WORKSPACE;
   int max_len = 0;
   for (int b = 0; b < g.B; ++b) {
-    if (h_len[b] < 1 || h_len[b] > g.cap) return QSA_ERR_INVALID_ARG;
+    if (h_len[b] < (shard ? 0 : 1) || h_len[b] > g.cap) return QSA_ERR_INVALID_ARG;
     max_len = std::max(max_len, h_len[b]);
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -809,7 +868,9 @@ qsa_status decode_impl(const void* q, const CacheView& view, const void* q_idx, 
   uint64_t* cand = reinterpret_cast<uint64_t*>(ws + g.o_cand);
   int32_t* rinfo = reinterpret_cast<int32_t*>(ws + g.o_rinfo);
   const int sms = num_sms();
-  const int max_nc_now = (max_len - 1) / 4;
+  // candidate blocks of the longest row: those before the query's own block, or for a shard
+  // at most every complete block it holds
+  const int max_nc_now = shard ? max_len / 4 : (max_len - 1) / 4;
   // the decode kernels form one chain of programmatic dependent launches (each waits for the
   // one before it); the first also follows the caller's last kernel (the append) that way
   {
@@ -855,6 +916,10 @@ qsa_status decode_impl(const void* q, const CacheView& view, const void* q_idx, 
     a.kbar_oob_row = static_cast<int32_t>(view.kbar_rows);
     a.n_c_out = n_c;
     a.hist = hist;
+    if (shard) {
+      a.glen = shard->glen;
+      a.block0 = shard->block0;
+    }
     a.w = reinterpret_cast<const __nv_bfloat16*>(w);
     a.scores = scores;
     a.ld = g.ld;
@@ -882,55 +947,25 @@ qsa_status decode_impl(const void* q, const CacheView& view, const void* q_idx, 
                              static_cast<const int32_t*>(cand_cnt),
                              static_cast<const uint64_t*>(cand),
                              static_cast<const int32_t*>(rinfo), idx, cnt,
-                             static_cast<const int32_t*>(cache->len), g.pl, plan));
+                             static_cast<const int32_t*>(cache->len), g.pl,
+                             shard ? nullptr : plan, shard ? shard->cand_score : nullptr,
+                             shard ? shard->block0 : 0));
   }
+  if (shard) return QSA_OK;   // a shard's selection stops at its candidates
   // a6: split attention + combine
   {
-    AttnMaps maps;
-    const uint64_t dq[3] = {128, 24, static_cast<uint64_t>(g.B)};
-    const uint64_t sq[2] = {256, 24 * 256};
-    const uint32_t bq[3] = {64, 12, 1};
-    if (!make_tmap(&maps.q, q, 3, dq, sq, bq)) return QSA_ERR_CUDA;
-    const uint64_t dkv[2] = {128, static_cast<uint64_t>(view.kv_rows)};
-    const uint64_t skv[1] = {256};
-    for (int j = 0; j < kNumBoxSizes; ++j) {
-      const uint32_t bkv[2] = {64, 4u << j};
-      if (!make_tmap(&maps.k[j], cache->k_blocks, 2, dkv, skv, bkv)) return QSA_ERR_CUDA;
-      if (!make_tmap(&maps.v[j], cache->v_blocks, 2, dkv, skv, bkv)) return QSA_ERR_CUDA;
-    }
-    {
-    const qsa_status pst = prepare_attention();
-    if (pst != QSA_OK) return pst;
-  }
-    AttnArgs a{};
-    if (view.kv_rows >= 0x7fffffffll) return QSA_ERR_UNSUPPORTED;
-    a.oob_row = static_cast<int32_t>(view.kv_rows);
-    a.pg = view.pg;
-    a.plan = plan;
-    a.pl = g.pl;
-    a.decode = 1;
-    a.splits = g.splits;
-    a.cap_blocks = g.cap / 4;
-    a.part_o = reinterpret_cast<float*>(ws + g.o_po);
-    a.part_m = reinterpret_cast<float*>(ws + g.o_pm);
-    a.part_l = reinterpret_cast<float*>(ws + g.o_pl);
-    a.st = dev_status(ws);
-    a.fault_tile = -1;
-    dim3 grid(g.B, 2, g.splits);
-    a.out = reinterpret_cast<__nv_bfloat16*>(out);   // written directly with one split
-    if (view.pg.table != nullptr) {
-      QSA_CHECK_PDL(launch_pdl(k_sparse_attn<true, true>, grid, dim3(AttnCfg::kThreads),
-                               AttnCfg::kSmemBytes, s, maps, a));
-    } else {
-      QSA_CHECK_PDL(launch_pdl(k_sparse_attn<true>, grid, dim3(AttnCfg::kThreads),
-                               AttnCfg::kSmemBytes, s, maps, a));
-    }
+    float* part_o = reinterpret_cast<float*>(ws + g.o_po);
+    float* part_m = reinterpret_cast<float*>(ws + g.o_pm);
+    float* part_l = reinterpret_cast<float*>(ws + g.o_pl);
+    st = launch_decode_attention(q, view, g, plan, dev_status(ws), out, g.splits, part_o, part_m,
+                                 part_l, false, s);
+    if (st != QSA_OK) return st;
     if (g.splits > 1) {
       const int warps = g.B * kHeads;
       QSA_CHECK_PDL(launch_pdl(k_decode_combine, dim3((warps * 32 + 255) / 256), dim3(256), 0, s,
-                               static_cast<const float*>(a.part_o),
-                               static_cast<const float*>(a.part_m),
-                               static_cast<const float*>(a.part_l), g.B, g.splits,
+                               static_cast<const float*>(part_o),
+                               static_cast<const float*>(part_m),
+                               static_cast<const float*>(part_l), g.B, g.splits,
                                reinterpret_cast<__nv_bfloat16*>(out)));
     }
   }
@@ -957,6 +992,82 @@ qsa_status qsa_decode_paged(const void* q, const qsa_paged_cache* cache, const v
   if (st != QSA_OK) return st;
   return decode_impl(q, view, q_idx, w, out, h_len, sel_idx, sel_cnt, workspace, ws_bytes, params,
                      stream);
+}
+
+// ---- context-sharded decode ---------------------------------------------------------------
+size_t qsa_decode_shard_workspace_size(const qsa_cache* shard, qsa_params params) {
+  return qsa_decode_workspace_size(shard, params);
+}
+
+qsa_status qsa_decode_shard_select(const void* q_idx, const void* w, const qsa_cache* shard,
+                                   int32_t block0, const int32_t* d_glen, const int32_t* h_len,
+                                   float* cand_score, int32_t* cand_idx, int32_t* cand_cnt,
+                                   void* workspace, size_t ws_bytes, qsa_params params,
+                                   qsa_stream_t stream) {
+  if (!shard) return QSA_ERR_INVALID_ARG;
+  ShardOpt o;
+  o.glen = d_glen;
+  o.block0 = block0;
+  o.cand_score = cand_score;
+  return decode_impl(nullptr, contiguous_view(shard), q_idx, w, nullptr, h_len, cand_idx,
+                     cand_cnt, workspace, ws_bytes, params, stream, &o);
+}
+
+qsa_status qsa_merge_candidates(const float* cand_score, const int32_t* cand_idx,
+                                const int32_t* cand_cnt, int32_t shards, int32_t batch,
+                                int32_t topk, int32_t max_blocks, int32_t* sel_idx,
+                                int32_t* sel_cnt, void* workspace, size_t ws_bytes,
+                                qsa_stream_t stream) {
+  qsa_status st = check_prefill_ptrs({cand_score, cand_idx, cand_cnt, sel_idx, sel_cnt, workspace});
+  if (st != QSA_OK) return st;
+  if (shards < 1 || shards > kMaxShards || batch < 1 || topk < 1 || topk > QSA_MAX_TOPK ||
+      max_blocks < 1 || max_blocks > QSA_MAX_SEQ_LEN / 4)
+    return QSA_ERR_INVALID_ARG;
+  if (ws_bytes < QSA_WS_HEADER_BYTES) return QSA_ERR_WORKSPACE;
+  const int nwords = (max_blocks + 31) / 32;
+  const int64_t smem = kTopkSharedBytes + int64_t(shards) * topk * 8 + 2 * int64_t(nwords) * 4;
+  if (smem > 227 * 1024) return QSA_ERR_UNSUPPORTED;
+  if (!set_smem(k_merge_candidates, static_cast<int>(smem))) return QSA_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  QSA_CHECK_PDL(launch_pdl(k_merge_candidates, dim3(batch), dim3(kTopkThreads),
+                           static_cast<size_t>(smem), s, cand_score, cand_idx, cand_cnt, shards,
+                           batch, topk, nwords, sel_idx, sel_cnt, dev_status(workspace)));
+  return QSA_OK;
+}
+
+qsa_status qsa_decode_shard_attend(const void* q, const qsa_cache* shard, int32_t block0,
+                                   const int32_t* d_glen, const int32_t* sel_idx,
+                                   const int32_t* sel_cnt, float* part_o, float* part_m,
+                                   float* part_l, void* workspace, size_t ws_bytes,
+                                   qsa_params params, qsa_stream_t stream) {
+  if (!shard) return QSA_ERR_INVALID_ARG;
+  qsa_status st = check_prefill_ptrs({q, shard->k_blocks, shard->v_blocks, d_glen, sel_idx,
+                                      sel_cnt, part_o, part_m, part_l, workspace});
+  if (st != QSA_OK) return st;
+  if (block0 < 0 || block0 % 128 != 0) return QSA_ERR_INVALID_ARG;
+  DecodeGeom g;
+  st = decode_geom(shard, params, &g);
+  if (st != QSA_OK) return st;
+  if (ws_bytes < g.total) return QSA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned char* ws = reinterpret_cast<unsigned char*>(workspace);
+  int32_t* plan = reinterpret_cast<int32_t*>(ws + g.o_plan);
+  QSA_CHECK_PDL(launch_pdl(k_shard_plan, dim3(g.B), dim3(kPlanThreads), 0, s, sel_idx, sel_cnt,
+                           g.topk, d_glen, block0, g.cap / 4, g.pl, plan, dev_status(ws)));
+  return launch_decode_attention(q, contiguous_view(shard), g, plan, dev_status(ws), nullptr, 1,
+                                 part_o, part_m, part_l, true, s);
+}
+
+qsa_status qsa_combine_partials(const float* part_o, const float* part_m, const float* part_l,
+                                int32_t shards, int32_t batch, void* out, qsa_stream_t stream) {
+  qsa_status st = check_prefill_ptrs({part_o, part_m, part_l, out});
+  if (st != QSA_OK) return st;
+  if (shards < 1 || batch < 1) return QSA_ERR_INVALID_ARG;
+  const int warps = batch * kHeads;
+  QSA_CHECK_PDL(launch_pdl(k_combine_shards, dim3((warps * 32 + 255) / 256), dim3(256), 0,
+                           reinterpret_cast<cudaStream_t>(stream), part_o, part_m, part_l, batch,
+                           shards, reinterpret_cast<__nv_bfloat16*>(out)));
+  return QSA_OK;
 }
 
 }  // extern "C"

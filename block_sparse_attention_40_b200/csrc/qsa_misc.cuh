@@ -733,31 +733,29 @@ __device__ __forceinline__ void topk_select_candidates(TopkShared& S, const uint
   __syncthreads();
   const int per = (nwords + kTopkThreads - 1) / kTopkThreads;
   const int w0 = tid * per, w1 = min(nwords, w0 + per);
-  // the need_eq lowest equal keys join the selection: prefix popcounts over eqb
+  // One block scan places everything: fewer than topk (<= 1024) keys lie above T, so a
+  // thread's count of them fits 11 bits, under its count of keys equal to T.  The need_eq
+  // lowest-index equal keys join the selection, which is emitted in ascending block order.
   {
-    int local = 0;
-    for (int w = w0; w < w1; ++w) local += __popc(eqb[w]);
-    int tot;
-    int before = block_excl_scan(local, S.sh, &tot);
+    int l_gt = 0, l_eq = 0;
     for (int w = w0; w < w1; ++w) {
-      uint32_t bits = eqb[w];
-      while (bits && before < need_eq) {
-        const uint32_t low = bits & (0u - bits);
-        sel[w] |= low;
-        bits ^= low;
-        ++before;
-      }
+      l_gt += __popc(sel[w]);
+      l_eq += __popc(eqb[w]);
     }
-  }
-  __syncthreads();
-  // ascending output: prefix popcounts over sel
-  {
-    int local = 0;
-    for (int w = w0; w < w1; ++w) local += __popc(sel[w]);
     int tot;
-    int pos = block_excl_scan(local, S.sh, &tot);
+    const int ex = block_excl_scan(l_eq * 2048 + l_gt, S.sh, &tot);
+    const int eq_before = ex >> 11, gt_before = ex & 2047;
+    int take = min(max(need_eq - eq_before, 0), l_eq);
+    int pos = gt_before + min(eq_before, need_eq);
     for (int w = w0; w < w1; ++w) {
       uint32_t bits = sel[w];
+      uint32_t e = eqb[w];
+      while (e && take > 0) {
+        const uint32_t low = e & (0u - e);
+        bits |= low;
+        e ^= low;
+        --take;
+      }
       while (bits) {
         const int b = __ffs(bits) - 1;
         bits &= bits - 1;
@@ -769,14 +767,33 @@ __device__ __forceinline__ void topk_select_candidates(TopkShared& S, const uint
   __syncthreads();   // S and the bitmaps are reused by the caller's next row
 }
 
+// What the finish kernel emits for a row once its k selected blocks are in out[0 .. k): the
+// attention plan record of the one-token tile, or (the decode of one shard of a longer
+// context, cand_score non-null) the (score, global block) candidates of the shard.
+__device__ __forceinline__ void finish_emit(int32_t* rec, const PlanLayout& pl, int32_t* out,
+                                            int k, int c, int p, const float* row_scores,
+                                            float* cand_score_row, int32_t block0) {
+  if (cand_score_row == nullptr) {
+    write_decode_plan(rec, pl, out, k, c, p);
+    return;
+  }
+  for (int j = threadIdx.x; j < k; j += blockDim.x) {
+    const int i = out[j];
+    cand_score_row[j] = row_scores[i];
+    out[j] = i + block0;
+  }
+}
+
 // Shared memory: TopkShared, then cap candidates (uint64), then two bitmaps of n_max bits.
-// Besides idx/cnt, the finish kernel writes each row's attention plan record (one-token tile).
+// Besides idx/cnt, the finish kernel writes each row's attention plan record (one-token tile),
+// or, for a shard (cand_score non-null), the selected blocks' scores and global block ids.
 __global__ void __launch_bounds__(kTopkThreads) k_topk_finish(
     const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_c, int topk,
     int cap, int n_max, const uint32_t* __restrict__ hist, const int32_t* __restrict__ cand_cnt,
     const uint64_t* __restrict__ cand, const int32_t* __restrict__ rinfo,
     int32_t* __restrict__ idx, int32_t* __restrict__ cnt, const int32_t* __restrict__ len,
-    PlanLayout pl, int32_t* __restrict__ plan) {
+    PlanLayout pl, int32_t* __restrict__ plan, float* __restrict__ cand_score,
+    int32_t block0) {
   pdl_trigger();
   pdl_wait();
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -789,13 +806,15 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk_finish(
   const int r = blockIdx.x;
   const int n = n_c[r];
   int32_t* out = idx + static_cast<int64_t>(r) * topk;
-  int32_t* rec = plan + static_cast<int64_t>(r) * pl.stride;
+  int32_t* rec = plan != nullptr ? plan + static_cast<int64_t>(r) * pl.stride : nullptr;
   const int p = len[r] - 1;
+  const float* row_scores = scores + static_cast<int64_t>(r) * ld;
+  float* cs = cand_score != nullptr ? cand_score + static_cast<int64_t>(r) * topk : nullptr;
   if (n <= topk) {
     for (int i = tid; i < topk; i += blockDim.x) out[i] = i < n ? i : -1;
     if (tid == 0) cnt[r] = n < 0 ? 0 : n;
     __syncthreads();
-    write_decode_plan(rec, pl, out, n < 0 ? 0 : n, n < 0 ? 0 : n, p);
+    finish_emit(rec, pl, out, n < 0 ? 0 : n, n < 0 ? 0 : n, p, row_scores, cs, block0);
     return;
   }
   const uint32_t* h = hist + static_cast<int64_t>(r) * 4096;
@@ -806,17 +825,17 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk_finish(
   const int C = cand_cnt[r];
   if (above + in_b1 > cap || C > cap) {
     // the candidates did not fit: full-row radix select on the scores in global memory
-    topk_row(scores + static_cast<int64_t>(r) * ld, n, topk, h, out, S);
+    topk_row(row_scores, n, topk, h, out, S);
     if (tid == 0) cnt[r] = topk;
     __syncthreads();
-    write_decode_plan(rec, pl, out, topk, n, p);
+    finish_emit(rec, pl, out, topk, n, p, row_scores, cs, block0);
     return;
   }
   for (int i = tid; i < C; i += blockDim.x) c[i] = cand[static_cast<int64_t>(r) * cap + i];
   topk_select_candidates(S, c, C, b1, topk - above, sel, eqb, (n + 31) / 32, topk, out);
   if (tid == 0) cnt[r] = topk;
   __syncthreads();
-  write_decode_plan(rec, pl, out, topk, n, p);
+  finish_emit(rec, pl, out, topk, n, p, row_scores, cs, block0);
 }
 
 // Step a3 on score rows, one CTA per row (grid-strided): pass 1 reads the row and builds the
@@ -1077,6 +1096,166 @@ __global__ void k_decode_combine(const float* __restrict__ part_o, const float* 
   pk.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
   pk.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
   reinterpret_cast<uint2*>(out + (static_cast<int64_t>(b) * kHeads + h) * kHeadDim)[lane] = pk;
+}
+
+// ---------------------------------------------------------------------------------------
+// Context-sharded decode.  A sequence's context is split over shards (caches of consecutive
+// tokens, each starting on a 512-token boundary, one per GPU); every shard proposes the top-k
+// of its own candidate blocks, and the selection is the top-k of their union.
+
+// Merge: the shards' (score, global block) candidates of one sequence -> the sequence's
+// selection, larger score first and the lower block among equal scores, emitted in ascending
+// block order (the same order as a selection over the whole context).  One CTA per sequence.
+// cs/ci [shards][batch][topk], cc [shards][batch].  Shared memory: TopkShared, then
+// shards * topk composites, then two bitmaps of nwords words (global blocks < 32 nwords).
+constexpr int kMaxShards = 64;
+__global__ void __launch_bounds__(kTopkThreads) k_merge_candidates(
+    const float* __restrict__ cs, const int32_t* __restrict__ ci, const int32_t* __restrict__ cc,
+    int shards, int batch, int topk, int nwords, int32_t* __restrict__ idx,
+    int32_t* __restrict__ cnt, DevStatus st) {
+  pdl_trigger();
+  pdl_wait();
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  TopkShared& S = *reinterpret_cast<TopkShared*>(smem_raw);
+  uint64_t* c = reinterpret_cast<uint64_t*>(smem_raw + kTopkSharedBytes);
+  uint32_t* sel = reinterpret_cast<uint32_t*>(c + static_cast<int64_t>(shards) * topk);
+  uint32_t* eqb = sel + nwords;
+  __shared__ int s_off[kMaxShards + 1];
+  const int b = blockIdx.x, tid = threadIdx.x;
+  if (tid == 0) {
+    int o = 0;
+    for (int r = 0; r < shards; ++r) {
+      s_off[r] = o;
+      int k = cc[static_cast<int64_t>(r) * batch + b];
+      if (k < 0 || k > topk) {
+        report_error(st, kErrDevice, 310);
+        k = k < 0 ? 0 : topk;
+      }
+      o += k;
+    }
+    s_off[shards] = o;
+  }
+  __syncthreads();
+  const int C = s_off[shards];
+  for (int r = 0; r < shards; ++r) {
+    const int k = s_off[r + 1] - s_off[r];
+    for (int j = tid; j < k; j += blockDim.x) {
+      const int64_t e = (static_cast<int64_t>(r) * batch + b) * topk + j;
+      int blk = ci[e];
+      uint32_t key = float_key(cs[e]);
+      if (blk < 0 || blk >= 32 * nwords) {   // never followed: reported, ranked last
+        report_error(st, kErrDevice, 311);
+        blk = 0;
+        key = 0u;
+      }
+      c[s_off[r] + j] = (static_cast<uint64_t>(key) << 32) | static_cast<uint32_t>(blk);
+    }
+  }
+  const int K = C < topk ? C : topk;
+  int32_t* out = idx + static_cast<int64_t>(b) * topk;
+  for (int j = K + tid; j < topk; j += blockDim.x) out[j] = -1;
+  if (tid == 0) cnt[b] = K;
+  if (K == 0) return;   // uniform
+  for (int i = tid; i < kTopkBins; i += blockDim.x) S.hist[i] = 0;
+  __syncthreads();
+  for (int i = tid; i < C; i += blockDim.x)
+    atomicAdd(&S.hist[static_cast<uint32_t>(c[i] >> 32) >> 20], 1u);
+  __syncthreads();
+  int above;
+  const uint32_t b1 = static_cast<uint32_t>(topk_find_bin(S, kTopkBins, K, &above));
+  topk_select_candidates(S, c, C, b1, K - above, sel, eqb, nwords, K, out);
+}
+
+// Attention plan of one shard (one-token tile per sequence): the selected blocks (ascending
+// global ids) that lie in the shard's blocks [block0, block0 + nblk), as local ids, followed by
+// the query's own block when the shard holds it; every union block is attended.  One CTA per
+// sequence.
+__global__ void __launch_bounds__(kPlanThreads) k_shard_plan(
+    const int32_t* __restrict__ sel_idx, const int32_t* __restrict__ sel_cnt, int topk,
+    const int32_t* __restrict__ glen, int32_t block0, int32_t nblk, PlanLayout pl,
+    int32_t* __restrict__ plan, DevStatus st) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ int s_lo, s_hi;
+  const int b = blockIdx.x, tid = threadIdx.x;
+  const int p = glen[b] - 1;
+  const int own = p >= 0 ? p / kBlock : -1;
+  int n = sel_cnt[b];
+  if (n < 0 || n > topk) {
+    if (tid == 0) report_error(st, kErrDevice, 312);
+    n = n < 0 ? 0 : topk;
+  }
+  const int32_t* s = sel_idx + static_cast<int64_t>(b) * topk;
+  if (tid == 0) {
+    int lo = 0, hi = n;   // first entry >= block0
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (s[mid] < block0) lo = mid + 1; else hi = mid;
+    }
+    int lo2 = lo, hi2 = n;   // first entry >= block0 + nblk
+    while (lo2 < hi2) {
+      const int mid = (lo2 + hi2) >> 1;
+      if (s[mid] < block0 + nblk) lo2 = mid + 1; else hi2 = mid;
+    }
+    s_lo = lo;
+    s_hi = lo2;
+  }
+  __syncthreads();
+  const int lo = s_lo, k = s_hi - s_lo;
+  const bool own_here = own >= block0 && own < block0 + nblk;
+  const int U = k + (own_here ? 1 : 0);
+  int32_t* rec = plan + static_cast<int64_t>(b) * pl.stride;
+  int32_t* uni = rec + pl.union_off();
+  for (int j = tid; j < k; j += blockDim.x) {
+    const int blk = s[lo + j];
+    if (blk >= own) report_error(st, kErrDevice, 313);   // not a candidate of the query
+    uni[j] = blk - block0;
+  }
+  uint32_t* m = reinterpret_cast<uint32_t*>(rec + pl.mask_off());
+  for (int q = tid; q < (U + 31) / 32; q += blockDim.x) {
+    const int rem = U - 32 * q;
+    m[q] = rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u);
+  }
+  if (tid == 0) {
+    if (own_here) uni[k] = own - block0;
+    rec[0] = U;
+    rec[1] = 1;
+    rec[2] = p;
+    rec[pl.tail_off()] = own_here ? k : -1000000;   // no own block here: nothing to hide
+  }
+}
+
+// Combine: the shards' partial softmaxes of every (sequence, head), by log-sum-exp.
+//   part_o [shards][B][24][128] (unnormalised, fp32), part_m (log2 domain), part_l
+//   [shards][B][24].  One warp per (sequence, head), 4 dims per lane.
+__global__ void k_combine_shards(const float* __restrict__ part_o, const float* __restrict__ part_m,
+                                 const float* __restrict__ part_l, int batch, int shards,
+                                 __nv_bfloat16* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= batch * kHeads) return;
+  const int64_t per_shard = static_cast<int64_t>(batch) * kHeads;
+  float M = -INFINITY;
+  for (int r = 0; r < shards; ++r) M = fmaxf(M, part_m[r * per_shard + warp]);
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  float L = 0.f;
+  for (int r = 0; r < shards; ++r) {
+    const float m = part_m[r * per_shard + warp];
+    const float f = (m == -INFINITY) ? 0.f : exp2f(m - M);
+    L += f * part_l[r * per_shard + warp];
+    const float4 o = reinterpret_cast<const float4*>(part_o + (r * per_shard + warp) * kHeadDim)[lane];
+    acc[0] += f * o.x;
+    acc[1] += f * o.y;
+    acc[2] += f * o.z;
+    acc[3] += f * o.w;
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  uint2 pk;
+  pk.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  pk.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+  reinterpret_cast<uint2*>(out + static_cast<int64_t>(warp) * kHeadDim)[lane] = pk;
 }
 
 }  // namespace qsa

@@ -62,6 +62,10 @@ struct ScoreArgs {
   Paging pg;               // where each sequence's compressed keys live (table null: contiguous)
   int32_t kbar_oob_row;    // a row past the compressed-key pool (TMA reads it as zeros)
   int32_t* n_c_out;        // [B] n_c per sequence (written by split 0), may be null
+  // decode of one shard of a longer context: the cache holds the sequence's tokens from
+  // global block block0 on, glen [B] holds the sequences' whole lengths (null: not a shard)
+  const int32_t* glen;
+  int32_t block0;
   uint32_t* hist;          // [B][4096] first-digit histograms of the scores (zeroed), or null
   // common
   const __nv_bfloat16* w;  // prefill: [T][16]; decode: [B][16]
@@ -80,6 +84,7 @@ struct ScoreWork {
   int32_t pos0;      // position (within the sequence) of token 0
   int64_t out_row0;  // score row of token 0
   int32_t seq;       // decode: the sequence
+  int32_t n_c;       // decode: candidate blocks (local to the cache) of the sequence
 };
 
 // s = sum_h w[h] * ReLU(d[h]) over the 16 heads of one (token, block): the even and the odd
@@ -126,11 +131,22 @@ __device__ __forceinline__ ScoreWork<NTOK> score_work(const ScoreArgs& a) {
     wk.b_row0 = static_cast<int32_t>((m.tok0 + p0) * kIdxHeads);
     wk.out_row0 = m.tok0 + p0 - a.row_begin;
     wk.seq = s;
+    wk.n_c = 0;   // per token: floor(pos / 4)
   } else {
     const int b = static_cast<int>(blockIdx.x) / a.splits;
     const int split = static_cast<int>(blockIdx.x) % a.splits;
-    const int p = a.len[b] - 1;
-    int n_c = p >= 0 ? p / kBlock : 0;
+    int p, n_c;
+    if (a.glen != nullptr) {
+      // a shard: the candidates are the shard's complete blocks before the query's own block
+      p = a.glen[b] - 1;
+      const int own = p >= 0 ? p / kBlock : 0;
+      n_c = own - a.block0;
+      const int here = a.len[b] / kBlock;
+      n_c = n_c < 0 ? 0 : (n_c > here ? here : n_c);
+    } else {
+      p = a.len[b] - 1;
+      n_c = p >= 0 ? p / kBlock : 0;
+    }
     // The grid covers the blocks of the host lengths the caller passed.  A device length
     // beyond them (a stale host copy) is reported, and only the covered blocks are scored;
     // the top-k then sees that same count, so it never reads a score that was not written.
@@ -152,6 +168,7 @@ __device__ __forceinline__ ScoreWork<NTOK> score_work(const ScoreArgs& a) {
     wk.b_row0 = b * kIdxHeads;
     wk.out_row0 = b;
     wk.seq = b;
+    wk.n_c = n_c;
   }
   return wk;
 }
@@ -243,6 +260,7 @@ __global__ void __launch_bounds__(ScoreCfg<NTOK>::kThreads, ScoreCfg<NTOK>::kCta
         }
         return wk.a_row0 + 128ll * m;
       };
+      const uint64_t pol_stream = l2_policy_evict_first();
       int64_t row_next = wk.n_mtiles > 0 ? tile_row(wk.mt0) : 0;
       for (int i = 0; i < wk.n_mtiles; ++i) {
         const int s = i % C::kStages;
@@ -250,7 +268,14 @@ __global__ void __launch_bounds__(ScoreCfg<NTOK>::kThreads, ScoreCfg<NTOK>::kCta
         if (i + 1 < wk.n_mtiles) row_next = tile_row(wk.mt0 + i + 1);
         if (!mbar_wait(&empty[s], ((i / C::kStages) & 1) ^ 1, s_abort, args.st, 10)) break;
         mbar_arrive_expect_tx(&full[s], C::kABytes);
-        tma_load_2d(sA + s * C::kABytes, &tmap_kbar, 0, static_cast<int32_t>(row), &full[s]);
+        if constexpr (NTOK == 1) {
+          // decode: the compressed keys are read once per step; keep the scores (written
+          // next, read back by the top-k) in L2 instead
+          tma_load_2d_hint(sA + s * C::kABytes, &tmap_kbar, 0, static_cast<int32_t>(row),
+                           &full[s], pol_stream);
+        } else {
+          tma_load_2d(sA + s * C::kABytes, &tmap_kbar, 0, static_cast<int32_t>(row), &full[s]);
+        }
         ++issued;
       }
       if (*s_abort) {
@@ -291,6 +316,7 @@ __global__ void __launch_bounds__(ScoreCfg<NTOK>::kThreads, ScoreCfg<NTOK>::kCta
     const int part = ew / 4;               // which group of four tokens (prefill)
     constexpr int kTokPerWarp = NTOK == 16 ? 4 : 1;
     const int tok_base = part * kTokPerWarp;
+    const uint64_t pol_keep = NTOK == 1 ? l2_policy_evict_last() : 0ull;
     for (int i = 0; i < wk.n_mtiles; ++i) {
       const int a = i % C::kNumAcc;
       const bool got = mbar_wait(&acc_full[a], (i / C::kNumAcc) & 1, s_abort, args.st, 14);
@@ -310,13 +336,21 @@ __global__ void __launch_bounds__(ScoreCfg<NTOK>::kThreads, ScoreCfg<NTOK>::kCta
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[a]);
       const int blk = 128 * (wk.mt0 + i) + quarter * 32 + lane;
+      float sc[kTokPerWarp];
+#pragma unroll
+      for (int j = 0; j < kTokPerWarp; ++j)
+        sc[j] = head_weighted_relu_sum(acc + j * kIdxHeads, sW + (tok_base + j) * kIdxHeads);
 #pragma unroll
       for (int j = 0; j < kTokPerWarp; ++j) {
         const int tok = tok_base + j;
-        const float s = head_weighted_relu_sum(acc + j * kIdxHeads, sW + tok * kIdxHeads);
+        const float s = sc[j];
         const int pos = wk.pos0 + tok;
-        const bool valid = tok < wk.ntok && blk < pos / kBlock;
-        if (valid) args.scores[(wk.out_row0 + tok) * args.ld + blk] = s;
+        const bool valid = tok < wk.ntok && blk < (NTOK == 1 ? wk.n_c : pos / kBlock);
+        if (valid) {
+          float* dst = args.scores + (wk.out_row0 + tok) * args.ld + blk;
+          if constexpr (NTOK == 1) st_global_hint(dst, s, pol_keep);
+          else *dst = s;
+        }
         if constexpr (NTOK == 1) {
           if (args.hist && valid) atomicAdd(&sHist[float_key(s) >> 20], 1u);
         }

@@ -237,6 +237,70 @@ QSA_API qsa_status qsa_decode(const void *q, const qsa_cache *cache, const void 
                       qsa_stream_t stream);
 
 /* ---------------------------------------------------------------------------------- */
+/* Context-sharded decode ("Long context became an architecture problem", section "Open
+ * weights still require a compatible runtime": 262,144 tokens native, extendable to one
+ * million; the pages describe no multi-GPU scheme, so the one below is this library's own).
+ * A batch's contexts are split over R shards, one per GPU: shard r is an ordinary qsa_cache
+ * (contiguous) holding tokens [t0_r, t0_r + capacity) of every sequence, with t0_r a multiple
+ * of 512 (block0 = t0_r / 4 is then a multiple of 128), shards back to back in token order.
+ * Its len[b] counts the tokens of sequence b stored there (0 .. capacity); every shard before
+ * the one holding a sequence's last token must be full.  Appends go with qsa_append_kv to the
+ * shard that holds the new token.  One decode step is then:
+ *   1. every shard: qsa_decode_shard_select -> its top-k (score, global block) candidates;
+ *   2. exchange: every rank gathers all shards' candidates (e.g. an NCCL all-gather);
+ *   3. every rank: qsa_merge_candidates -> the selection (identical on every rank, and bit
+ *      for bit the selection qsa_decode would make over the whole context);
+ *   4. every shard: qsa_decode_shard_attend -> per-(sequence, head) partial softmax over the
+ *      selected blocks it holds (plus the query's own block on the shard that holds it);
+ *   5. exchange the partials, then qsa_combine_partials -> the output.
+ * d_glen: int32 [batch] device, the sequences' whole lengths (after the append).  The
+ * workspace of a shard call is qsa_decode_shard_workspace_size(shard) bytes (the decode
+ * workspace of that cache). */
+QSA_API size_t qsa_decode_shard_workspace_size(const qsa_cache *shard, qsa_params params);
+
+/*   q_idx bf16 [batch][16][64], w bf16 [batch][16]: the decode query's indexer inputs.
+ *   h_len int32 [batch] HOST copy of shard->len (sizes the grids).
+ *   cand_score fp32 [batch][topk], cand_idx int32 [batch][topk], cand_cnt int32 [batch]:
+ *   the shard's min(topk, n) best candidate blocks (global ids, ascending; padded with -1)
+ *   and their scores, n = its complete blocks before the query's own block. */
+QSA_API qsa_status qsa_decode_shard_select(const void *q_idx, const void *w,
+                                           const qsa_cache *shard, int32_t block0,
+                                           const int32_t *d_glen, const int32_t *h_len,
+                                           float *cand_score, int32_t *cand_idx,
+                                           int32_t *cand_cnt, void *workspace, size_t ws_bytes,
+                                           qsa_params params, qsa_stream_t stream);
+
+/* cand_score fp32 [shards][batch][topk], cand_idx int32 [shards][batch][topk], cand_cnt int32
+ * [shards][batch] (the shards' outputs stacked in shard order); max_blocks > every global
+ * block id (the whole capacity / 4).  sel_idx int32 [batch][topk] (ascending, -1 padded) and
+ * sel_cnt int32 [batch] receive the selection: the topk best of all candidates, larger score
+ * first and the lower block among equal scores.  shards <= 64; the call needs
+ * shards * topk * 8 + max_blocks / 4 bytes of shared memory (about 200 KB at most), else
+ * QSA_ERR_UNSUPPORTED.  workspace: at least QSA_WS_HEADER_BYTES (device status only). */
+QSA_API qsa_status qsa_merge_candidates(const float *cand_score, const int32_t *cand_idx,
+                                        const int32_t *cand_cnt, int32_t shards, int32_t batch,
+                                        int32_t topk, int32_t max_blocks, int32_t *sel_idx,
+                                        int32_t *sel_cnt, void *workspace, size_t ws_bytes,
+                                        qsa_stream_t stream);
+
+/*   q bf16 [batch][24][128]; sel_idx/sel_cnt as returned by qsa_merge_candidates.
+ *   part_o fp32 [batch][24][128] (unnormalised), part_m fp32 [batch][24] (running max, in
+ *   log2 units of the scaled scores), part_l fp32 [batch][24] (sum of exponentials): this
+ *   shard's part of the softmax (m = -inf, l = 0, o = 0 when it holds none of the keys). */
+QSA_API qsa_status qsa_decode_shard_attend(const void *q, const qsa_cache *shard,
+                                           int32_t block0, const int32_t *d_glen,
+                                           const int32_t *sel_idx, const int32_t *sel_cnt,
+                                           float *part_o, float *part_m, float *part_l,
+                                           void *workspace, size_t ws_bytes, qsa_params params,
+                                           qsa_stream_t stream);
+
+/* part_o fp32 [shards][batch][24][128], part_m / part_l fp32 [shards][batch][24] (stacked in
+ * shard order) -> out bf16 [batch][24][128], merged by log-sum-exp. */
+QSA_API qsa_status qsa_combine_partials(const float *part_o, const float *part_m,
+                                        const float *part_l, int32_t shards, int32_t batch,
+                                        void *out, qsa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------- */
 /* Decode without a caller-provided workspace.  The pages have no counterpart of this entry
  * point; it exists for callers that cannot allocate device memory on the call path and have
  * no buffer to lend -- for example a plugin running inside a host framework whose allocator

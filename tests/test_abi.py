@@ -145,3 +145,41 @@ def test_paged_cache_host_side_checks():
                              _p(good), _p(good), _p(good), h_len, None, None, _p(good), 1 << 30,
                              B._params(16), None)
     assert B.STATUS[r] == "QSA_ERR_INVALID_ARG"
+
+
+def test_sharded_decode_host_side_checks():
+    # shard entry points refuse bad geometry before anything is enqueued (no GPU needed)
+    lib = qsa.load()
+    good = 0x10000
+    prm = B._params(512)
+    desc = B.CacheDesc(good, good, good, good, good, 4, 262144)
+    h_len = (ctypes.c_int32 * 4)(*([1000] * 4))
+    assert lib.qsa_decode_shard_workspace_size(ctypes.byref(desc), prm) == \
+        lib.qsa_decode_workspace_size(ctypes.byref(desc), prm) > 0
+    for block0 in (100, -128):   # shards start on 512-token (128-block) boundaries
+        r = lib.qsa_decode_shard_select(_p(good), _p(good), ctypes.byref(desc), block0, _p(good),
+                                        h_len, _p(good), _p(good), _p(good), _p(good), 1 << 30,
+                                        prm, None)
+        assert B.STATUS[r] == "QSA_ERR_INVALID_ARG"
+        r = lib.qsa_decode_shard_attend(_p(good), ctypes.byref(desc), block0, _p(good), _p(good),
+                                        _p(good), _p(good), _p(good), _p(good), _p(good), 1 << 30,
+                                        prm, None)
+        assert B.STATUS[r] == "QSA_ERR_INVALID_ARG"
+    r = lib.qsa_decode_shard_select(_p(good + 4), _p(good), ctypes.byref(desc), 0, _p(good),
+                                    h_len, _p(good), _p(good), _p(good), _p(good), 1 << 30, prm,
+                                    None)
+    assert B.STATUS[r] == "QSA_ERR_ALIGNMENT"
+    # merge: shard count, budget and block range; too many candidates for shared memory
+    for shards, k, nblk, want in ((0, 512, 1024, "QSA_ERR_INVALID_ARG"),
+                                  (65, 512, 1024, "QSA_ERR_INVALID_ARG"),
+                                  (4, 0, 1024, "QSA_ERR_INVALID_ARG"),
+                                  (4, 512, 0, "QSA_ERR_INVALID_ARG"),
+                                  (64, 1024, 262144, "QSA_ERR_UNSUPPORTED")):
+        r = lib.qsa_merge_candidates(_p(good), _p(good), _p(good), shards, 4, k, nblk, _p(good),
+                                     _p(good), _p(good), 1 << 20, None)
+        assert B.STATUS[r] == want, (shards, k, nblk)
+    r = lib.qsa_merge_candidates(_p(good), _p(good), _p(good), 4, 4, 512, 1024, _p(good),
+                                 _p(good), _p(good), 16, None)
+    assert B.STATUS[r] == "QSA_ERR_WORKSPACE"
+    r = lib.qsa_combine_partials(_p(good), _p(good), _p(good), 0, 4, _p(good), None)
+    assert B.STATUS[r] == "QSA_ERR_INVALID_ARG"
