@@ -12,7 +12,8 @@
 //   softmax          one thread per row: keys of blocks the row's token did not select get
 //                    -inf (a per-block bias), and so do the own block's future tokens; online
 //                    max in the log2 domain with lazy rescaling of O (only when the max grows
-//                    by more than 2^8); P = exp2(.) written back over S in TMEM as bf16
+//                    by more than 2^8); P = exp2(.) as bf16 into its own TMEM columns, except
+//                    for pairs of blocks that no row of the warp attends, whose P is zero
 //   O += P V         tcgen05, A = P (TMEM), B = V chunk (smem, MN-major), D = O in TMEM;
 //                    its completion frees the V slot
 // Decode (kDec, one query token, 12 valid rows): the 12 head rows are loaded into each of the
@@ -40,9 +41,6 @@ namespace qsa {
 
 #ifndef QSA_ATTN_SOFT_GROUPS
 #define QSA_ATTN_SOFT_GROUPS 2
-#endif
-#ifndef QSA_ATTN_SKIP_BLOCKS
-#define QSA_ATTN_SKIP_BLOCKS 4   // prefill softmax: blocks per warp-uniform skip decision
 #endif
 struct AttnCfg {
   static constexpr int kSoftGroups = QSA_ATTN_SOFT_GROUPS;   // softmax warpgroups (2 or 4)
@@ -348,7 +346,6 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
   const int mwords = args.pl.umax / 32;
   const int col0 = kDec ? 0 : g * kHeadDim;
   // P: written over S in prefill; in its own columns [384, 512) in decode
-  // P (bf16, two per column) in its own columns: [384, 448) and [448, 512) for the two buffers
   const uint32_t tmem_P = tmem + 384;
   constexpr int kPStride = 64;
 
@@ -413,10 +410,10 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
         const int ks = i % C::kKStages;
         if (!mbar_wait(&k_full[ks], (i / C::kKStages) & 1, s_abort, args.st, 23, lim)) break;
         // S_i overwrites S_{i-2}, which the softmax finished reading before it arrived on
-        // p_full for chunk i-2 (waited for when P_{i-2}.V was issued).  P has its own
-        // columns, which no S MMA touches; the softmax rewrites P of this buffer only after
-        // s_full of chunk i, whose commit also covers P_{i-2}.V.  Decode keeps the older,
-        // stricter order (S_i after P_{i-2}.V has completed).
+        // p_full for chunk i-2 (waited for when P_{i-2}.V was issued).  P has its own columns,
+        // which no S MMA touches; the softmax rewrites P of this buffer only after s_full of
+        // chunk i, whose commit also covers P_{i-2}.V.  Decode keeps the stricter order (S_i
+        // after P_{i-2}.V has completed).
         if (kDec && i >= 2 && !mbar_wait(&p_free[b], ((i - 2) >> 1) & 1, s_abort, args.st, 29, lim))
           break;
         tc_fence_after();
@@ -631,28 +628,25 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
         }
       }
     } else {
-      // ---------------- prefill softmax (warps 0 .. 7) ----------------
-      // Two warpgroups share each row: group wg handles keys 64wg..64wg+63 (blocks
-      // 16wg..16wg+15) of every chunk and dims 64wg.. of O.  A warp's 32 rows belong to about
-      // three tokens, and each group of kSkipBlk blocks that none of them attends is skipped
-      // (a warp-uniform branch): no maximum, no exponentials, its P stays zero.  On long rows
-      // about half of the union's blocks are skipped so.  P (bf16 pairs) has its own TMEM
-      // columns, so S stays in TMEM until the S MMA of chunk i+2: the softmax reads it twice,
-      // 32 keys at a time (for the maximum, then for the exponentials), and keeps only the
-      // running statistics and the packed P in registers.  A row's unselected keys are dropped
-      // per block: out of the maximum, and through a -inf offset in the exponent.  Row maxima
-      // are exchanged between the two groups through shared memory (double-buffered by chunk
-      // parity, one named barrier per chunk); partial row sums are combined once at the end.
-      // Both groups take identical rescale decisions.
+      // ---------------- softmax (warps 0 .. 4 kSoftGroups - 1) ----------------
+      // kSoftGroups warpgroups share each row: group sg handles keys [kCols sg, kCols (sg + 1))
+      // of every chunk and dims [kCols sg, ...) of O.  Row maxima are exchanged through shared
+      // memory (double-buffered by chunk parity, one named barrier per chunk); partial row sums
+      // are combined once at the end.  All groups take identical rescale decisions.
+      // A warp's 32 rows belong to about three tokens: the exponentials of each pair of blocks
+      // that none of them attends are skipped (a warp-uniform branch) and its P is left zero,
+      // about half of the union's blocks on long rows.  The masking and the maximum still run
+      // over every key (skipping them too measured no faster).
       static_assert(C::kSoftGroups == 2, "prefill softmax assumes two warpgroups");
-      constexpr int kSkipBlk = QSA_ATTN_SKIP_BLOCKS;   // blocks per skip decision (2, 4 or 8)
-      static_assert(kSkipBlk == 2 || kSkipBlk == 4 || kSkipBlk == 8, "skip group of 2, 4 or 8");
-      constexpr uint32_t kGrpMask = (1u << kSkipBlk) - 1u;
+      constexpr int kSG = C::kSoftGroups;
+      constexpr int kCols = 128 / kSG;              // keys (and O dims) per group
+      constexpr int kBlk = kCols / kBlock;          // blocks per group
       const int wg = warp >> 2;
       const int quarter = warp & 3;           // TMEM lanes 32q .. 32q+31
       const int row = quarter * 32 + lane;
       const int valid_rows = kGroup * ntok;
       const bool row_ok = row < valid_rows;
+      const bool warp_active = quarter * 32 < valid_rows;
       const int tr = row_ok ? row / kGroup : 0;
       const int hr = row % kGroup;
       const int pos = pos0 + tr;
@@ -667,53 +661,55 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
       for (int i = 0; i < nchunks; ++i) {
         const int b = i & 1;
         const int q = c_begin + i;
-        const uint32_t mine = (mword_next >> (16 * wg)) & 0xffffu;   // my row's blocks
+        const uint32_t mword = (mword_next >> (kBlk * wg)) & ((1u << kBlk) - 1u);   // my blocks
+        const uint32_t warp_need = __reduce_or_sync(0xffffffffu, mword);   // blocks any row of the warp attends
         if (row_ok && i + 1 < nchunks) mword_next = mrow[q + 1];
-        const uint32_t need = __reduce_or_sync(0xffffffffu, mine);   // the warp's blocks
-        const int tu = tail_u - q * C::kChunkBlocks - 16 * wg;       // my own block, if here
-        const bool own_here = __any_sync(0xffffffffu, tu >= 0 && tu < 16);
         bool got = ok ? mbar_wait(&s_full[b], (i >> 1) & 1, s_abort, args.st, 24) : false;
         if (__any_sync(0xffffffffu, !got)) ok = false;   // also reconverges the warp
         tc_fence_after();
-        const uint32_t ts = tmem + lane_base + b * 128 + 64 * wg;
+        uint32_t sv[kCols];
+        const uint32_t ts = tmem + lane_base + b * 128;
         float mx = -INFINITY;
-        if (ok && need != 0u) {
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {   // keys 32h .. 32h+31 of my half: blocks 8h .. 8h+7
-            if ((need >> (8 * h)) & 0xffu) {
-              uint32_t sv[32];
-              tmem_ld32(ts + 32 * h, sv);
-              tmem_wait_ld();
-#pragma unroll
-              for (int gi = 0; gi < 8 / kSkipBlk; ++gi) {
-                const int u0 = 8 * h + gi * kSkipBlk;
-                if ((need >> u0) & kGrpMask) {
-#pragma unroll
-                  for (int ub = 0; ub < kSkipBlk; ++ub) {
-                    const int u = u0 + ub;
-                    const uint32_t* x = sv + 4 * (u - 8 * h);
-                    float k1 = __uint_as_float(x[1]), k2 = __uint_as_float(x[2]),
-                          k3 = __uint_as_float(x[3]);
-                    if (own_here && u == tu) {   // hide the tokens after the query
-                      if (tail_last < 1) k1 = -INFINITY;
-                      if (tail_last < 2) k2 = -INFINITY;
-                      if (tail_last < 3) k3 = -INFINITY;
-                    }
-                    const float m4 = fmaxf(fmaxf(__uint_as_float(x[0]), k1), fmaxf(k2, k3));
-                    if ((mine >> u) & 1u) mx = fmaxf(mx, m4);
-                  }
-                }
+        if (ok && warp_active) {
+  #pragma unroll
+          for (int c = 0; c < kCols / 32; ++c) tmem_ld32(ts + kCols * wg + 32 * c, sv + 32 * c);
+          tmem_wait_ld();
+          // keys of blocks this row's token did not select -> -inf
+  #pragma unroll
+          for (int u = 0; u < kBlk; ++u) {
+            const float bias = ((mword >> u) & 1u) ? 0.f : -INFINITY;
+  #pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              sv[4 * u + kk] = __float_as_uint(__uint_as_float(sv[4 * u + kk]) + bias);
+          }
+          // the own block: hide the tokens after the query (only where it lies)
+          const int tu = tail_u - q * C::kChunkBlocks - kBlk * wg;
+          if (__any_sync(0xffffffffu, tu >= 0 && tu < kBlk)) {
+  #pragma unroll
+            for (int u = 0; u < kBlk; ++u) {
+              if (u == tu) {
+                if (tail_last < 1) sv[4 * u + 1] = __float_as_uint(-INFINITY);
+                if (tail_last < 2) sv[4 * u + 2] = __float_as_uint(-INFINITY);
+                if (tail_last < 3) sv[4 * u + 3] = __float_as_uint(-INFINITY);
               }
             }
           }
+          float mxs[8];
+  #pragma unroll
+          for (int j = 0; j < 8; ++j) mxs[j] = __uint_as_float(sv[j]);
+  #pragma unroll
+          for (int j = 8; j < kCols; ++j) mxs[j & 7] = fmaxf(mxs[j & 7], __uint_as_float(sv[j]));
+          mx = fmaxf(fmaxf(fmaxf(mxs[0], mxs[1]), fmaxf(mxs[2], mxs[3])),
+                     fmaxf(fmaxf(mxs[4], mxs[5]), fmaxf(mxs[6], mxs[7])));
         }
-        // exchange the partial row maxima (every softmax warp takes part)
-        xmax[(b * 2 + wg) * 128 + row] = mx;
+        // exchange the partial row maxima (every softmax warp takes part, active or not)
+        xmax[(b * kSG + wg) * 128 + row] = mx;
         tc_fence_before();
-        named_barrier_sync(1, 256);
+        named_barrier_sync(1, 128 * kSG);
         tc_fence_after();
-        if (ok) {
-          mx = fmaxf(mx, xmax[(b * 2 + (wg ^ 1)) * 128 + row]);
+        if (ok && warp_active) {
+  #pragma unroll
+          for (int o = 1; o < kSG; ++o) mx = fmaxf(mx, xmax[(b * kSG + ((wg + o) % kSG)) * 128 + row]);
           const float m_cand = fmaxf(m, mx * sl2);
           const bool grow = m_cand > m + 8.f || (m == -INFINITY && m_cand > -INFINITY);
           const bool rescale = __any_sync(0xffffffffu, grow);
@@ -723,54 +719,30 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
             m = m_cand;
           }
           const float mneg = (m == -INFINITY) ? 0.f : -m;
-          uint32_t pv[32];   // P of my 64 keys, bf16 pairs; skipped groups stay zero
-          float lsum[2] = {0.f, 0.f};
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            if ((need >> (8 * h)) & 0xffu) {
-              uint32_t sv[32];
-              tmem_ld32(ts + 32 * h, sv);
-              tmem_wait_ld();
-#pragma unroll
-              for (int gi = 0; gi < 8 / kSkipBlk; ++gi) {
-                const int u0 = 8 * h + gi * kSkipBlk;
-                if ((need >> u0) & kGrpMask) {
-#pragma unroll
-                  for (int ub = 0; ub < kSkipBlk; ++ub) {
-                    const int u = u0 + ub;
-                    const uint32_t* x = sv + 4 * (u - 8 * h);
-                    // an unselected block: every exponent is -inf
-                    const float off = ((mine >> u) & 1u) ? mneg : -INFINITY;
-                    float p0 = ex2_approx(fmaf(__uint_as_float(x[0]), sl2, off));
-                    float p1 = ex2_approx(fmaf(__uint_as_float(x[1]), sl2, off));
-                    float p2 = ex2_approx(fmaf(__uint_as_float(x[2]), sl2, off));
-                    float p3 = ex2_approx(fmaf(__uint_as_float(x[3]), sl2, off));
-                    if (own_here && u == tu) {
-                      if (tail_last < 1) p1 = 0.f;
-                      if (tail_last < 2) p2 = 0.f;
-                      if (tail_last < 3) p3 = 0.f;
-                    }
-                    lsum[ub & 1] += (p0 + p1) + (p2 + p3);
-                    pv[2 * u] = pack_bf16x2(p0, p1);
-                    pv[2 * u + 1] = pack_bf16x2(p2, p3);
-                  }
-                } else {
-#pragma unroll
-                  for (int ub = 0; ub < kSkipBlk; ++ub) {
-                    pv[2 * (u0 + ub)] = 0u;
-                    pv[2 * (u0 + ub) + 1] = 0u;
-                  }
-                }
+          // P overwrites S in registers: packed pair j lands in sv[j], whose S value (key j) was
+          // consumed at pair j/2 <= j
+          float lsum[4] = {0.f, 0.f, 0.f, 0.f};
+          constexpr int kSk = 2;                 // blocks per skip decision (1, 2, 4: 2 measured best)
+  #pragma unroll
+          for (int gi = 0; gi < kBlk / kSk; ++gi) {
+            if ((warp_need >> (gi * kSk)) & ((1u << kSk) - 1u)) {
+  #pragma unroll
+              for (int jj = 0; jj < 2 * kSk; ++jj) {
+                const int j = gi * 2 * kSk + jj;
+                const float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * j]), sl2, mneg));
+                const float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * j + 1]), sl2, mneg));
+                lsum[j & 3] += p0 + p1;
+                sv[j] = pack_bf16x2(p0, p1);
               }
             } else {
-#pragma unroll
-              for (int j = 0; j < 16; ++j) pv[16 * h + j] = 0u;
+  #pragma unroll
+              for (int jj = 0; jj < 2 * kSk; ++jj) sv[gi * 2 * kSk + jj] = 0u;
             }
           }
-          l = l * alpha + (lsum[0] + lsum[1]);
-          // P of this buffer was last read by P.V of chunk i-2, which completed before S_i
-          // (one commit tracks every earlier MMA)
-          tmem_st32(tmem_P + lane_base + b * kPStride + 32 * wg, pv);
+          l = l * alpha + ((lsum[0] + lsum[1]) + (lsum[2] + lsum[3]));
+          // packed P of my keys -> columns kCols/2 sg .. of this buffer's P (P.V of chunk i-2,
+          // which last read them, completed before S_i: one commit tracks every earlier MMA)
+          tmem_st32(tmem_P + lane_base + b * kPStride + 32 * wg, sv);
           tmem_wait_st();
           if (rescale && i > 0) {
             // O holds P.V of chunks < i-1 and maybe i-1: wait until chunk i-1 is in, rescale
@@ -779,13 +751,13 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
             if (__any_sync(0xffffffffu, !gotpv)) ok = false;
             if (ok) {
               tc_fence_after();
-              const uint32_t to = tmem_O + lane_base + 64 * wg;
-#pragma unroll
-              for (int c = 0; c < 2; ++c) {
+              const uint32_t to = tmem_O + lane_base + kCols * wg;
+  #pragma unroll
+              for (int c = 0; c < kCols / 32; ++c) {
                 uint32_t ov[32];
                 tmem_ld32(to + 32 * c, ov);
                 tmem_wait_ld();
-#pragma unroll
+  #pragma unroll
                 for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
                 tmem_st32(to + 32 * c, ov);
               }
@@ -798,11 +770,11 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
         if (lane == 0) mbar_arrive(&p_full[b]);
       }
       // combine the partial row sums
-      constexpr int kCols = 64;   // O dims per group
-      const bool warp_active = quarter * 32 < valid_rows;
       xsum[wg * 128 + row] = l;
-      named_barrier_sync(1, 256);
-      const float l_all = xsum[row] + xsum[128 + row];
+      named_barrier_sync(1, 128 * kSG);
+      float l_all = 0.f;
+  #pragma unroll
+      for (int o = 0; o < kSG; ++o) l_all += xsum[o * 128 + row];
       if (ok && nchunks > 0) {
         // a dedicated barrier: two P.V may still be in flight here, so a parity wait on
         // pv_done could match an older phase
