@@ -38,18 +38,34 @@ DEC_BATCH, DEC_CAP = 64, 262144
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the roofline kernels from one
 # ncu capture: bytes per unit of work (prefill attention: per query token; decode step: per
-# sequence), the SHA-256 of the kernel sources the capture ran, and what was captured.  A
+# sequence), the SHA-256 of the sources in TRAFFIC_SOURCES at the capture, and what was captured.  A
 # figure is reported only while the sources are unchanged; otherwise the roofline's
 # "traffic" is null until a new capture is taken.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # 313,847,552 B read + 175,275,008 B written by one 32K-token prefill attention launch
+    # (profiles/k_sparse_attn_prefill_32k.md), per token; the attention's bytes (Q, O, the
+    # gathered K/V tiles, the plan) grow with the tokens of the launch.
+    "prefill_attention": (489122560 / 32768,
+                          "e3fdee859df326087c01791e2f3f71fb23768b6d5eda08d98bfbbb4ab0c32fd7",
+                          "ncu dram__bytes_read.sum + dram__bytes_write.sum of one 32K-token "
+                          "launch (profiles/k_sparse_attn_prefill_32k.md), scaled by tokens"),
+}
 
 
-def csrc_sha():
+# The sources each roofline kernel's code and launch depend on; a capture is stale once any
+# of them changes.
+TRAFFIC_SOURCES = {
+    "prefill_attention": ("qsa_attn.cuh", "qsa_common.cuh", "qsa_api.cu"),
+    "decode_step": None,   # the whole step: every source
+}
+
+
+def csrc_sha(files=None):
     import hashlib
     d = os.path.join(ROOT, "block_sparse_attention_40_b200", "csrc")
     h = hashlib.sha256()
     for n in sorted(os.listdir(d)):
-        if n.endswith((".cu", ".cuh")):
+        if n.endswith((".cu", ".cuh")) and (files is None or n in files):
             h.update(n.encode())
             h.update(open(os.path.join(d, n), "rb").read())
     return h.hexdigest()
@@ -61,7 +77,7 @@ def measured_traffic(kernel, units):
     if rec is None:
         return None, "no ncu capture of the current kernel"
     per_unit, sha, what = rec
-    if sha != csrc_sha():
+    if sha != csrc_sha(TRAFFIC_SOURCES[kernel]):
         return None, "kernel sources changed since the ncu capture"
     return per_unit * units, what
 

@@ -58,6 +58,31 @@ __device__ __forceinline__ int block_excl_scan(int v, int* sh /*[33]*/, int* tot
   return excl;
 }
 
+// The same scan with one barrier: every warp reads all warp totals and scans them itself.
+// sh[0 .. warps) is written before the barrier and read after it, so the caller must pass at
+// least one more __syncthreads before sh is written again (the next call included).
+__device__ __forceinline__ int block_excl_scan_1bar(int v, int* sh /*[32]*/, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nw = (blockDim.x + 31) >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sh[warp] = x;
+  __syncthreads();
+  int t = lane < nw ? sh[lane] : 0;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, t, o);
+    if (lane >= o) t += y;
+  }
+  const int before = __shfl_sync(0xffffffffu, t, (warp + 31) & 31);   // inclusive, warp - 1
+  *total = __shfl_sync(0xffffffffu, t, nw - 1);
+  return x - v + (warp > 0 ? before : 0);
+}
+
 // One CTA: metadata for every sequence (prefix sums over blocks and tiles).
 __global__ void __launch_bounds__(1024) k_seq_meta(const int32_t* __restrict__ cu, int num_seqs,
                                                    int rows_per_tile, SeqMeta* __restrict__ meta,
@@ -429,8 +454,9 @@ constexpr int kTopkBins = 4096;
 
 struct TopkShared {
   uint32_t hist[kTopkBins];
+  uint32_t hist3[256];   // third digit of the candidate select, cleared with the second's
   int sh[40];
-  int sel[2];
+  int sel[4];   // threshold bin, keys above it, keys in it
   int wgt[kTopkWarps];
   int weq[kTopkWarps];
 };
@@ -438,36 +464,59 @@ struct TopkShared {
 // the float4 copy; the host sizes the allocation with the same constant).
 constexpr int kTopkSharedBytes = (static_cast<int>(sizeof(TopkShared)) + 127) / 128 * 128;
 
-// Find the bin where the count of keys in higher bins first reaches `need` (bins scanned
-// from the top).  Returns the bin; *above receives the count of keys in higher bins.
-__device__ __forceinline__ int topk_find_bin(TopkShared& S, int nbins, int need, int* above) {
+// Find the bin of `hist` where the count of keys in higher bins first reaches `need` (bins
+// scanned from the top).  Returns the bin; *above receives the count of keys in higher bins and
+// *in_bin (if given) the bin's own count.  nbins is kTopkBins (eight bins a thread, read as
+// two uint4, thread 0 holding the highest) or at most kTopkThreads (one bin a thread).  One
+// block scan places every thread's bins; only the thread whose range holds the crossing walks
+// its bins.  Two barriers; the histogram may be rewritten as soon as this returns.
+static_assert(kTopkBins == 8 * kTopkThreads, "topk_find_bin holds eight bins a thread");
+__device__ __forceinline__ int topk_find_bin(TopkShared& S, const uint32_t* hist, int nbins,
+                                             int need, int* above, int* in_bin = nullptr) {
   const int tid = threadIdx.x;
-  const int per = nbins / kTopkThreads;   // 8 or 1 (or 0: only the first threads)
-  int local = 0;
-  int lo_bin = 0, hi_bin = -1;
-  if (per > 0) {
-    hi_bin = nbins - 1 - tid * per;       // thread 0 owns the highest bins
-    lo_bin = hi_bin - per + 1;
-  } else if (tid < nbins) {
-    hi_bin = lo_bin = nbins - 1 - tid;
-  }
-  for (int b = hi_bin; b >= lo_bin; --b) local += static_cast<int>(S.hist[b]);
   int tot;
-  const int ex = block_excl_scan(local, S.sh, &tot);   // keys in bins above my range
-  int running = ex;
-  for (int b = hi_bin; b >= lo_bin; --b) {
-    const int h = static_cast<int>(S.hist[b]);
-    if (running < need && running + h >= need) {
-      S.sel[0] = b;
-      S.sel[1] = running;
+  if (nbins == kTopkBins) {
+    const int lo = kTopkBins - 8 * (tid + 1);
+    const uint4 h0 = *reinterpret_cast<const uint4*>(hist + lo);
+    const uint4 h1 = *reinterpret_cast<const uint4*>(hist + lo + 4);
+    const int v[8] = {static_cast<int>(h0.x), static_cast<int>(h0.y), static_cast<int>(h0.z),
+                      static_cast<int>(h0.w), static_cast<int>(h1.x), static_cast<int>(h1.y),
+                      static_cast<int>(h1.z), static_cast<int>(h1.w)};
+    int local = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) local += v[j];
+    int running = block_excl_scan_1bar(local, S.sh, &tot);   // keys in bins above my range
+    if (running < need && running + local >= need) {
+#pragma unroll
+      for (int j = 7; j >= 0; --j) {
+        if (running < need && running + v[j] >= need) {
+          S.sel[0] = lo + j;
+          S.sel[1] = running;
+          S.sel[2] = v[j];
+        }
+        running += v[j];
+      }
     }
-    running += h;
+  } else {
+    const int bin = nbins - 1 - tid;
+    const int c = bin >= 0 ? static_cast<int>(hist[bin]) : 0;
+    const int running = block_excl_scan_1bar(c, S.sh, &tot);
+    if (bin >= 0 && running < need && running + c >= need) {
+      S.sel[0] = bin;
+      S.sel[1] = running;
+      S.sel[2] = c;
+    }
   }
   __syncthreads();
   *above = S.sel[1];
-  const int bin = S.sel[0];
-  __syncthreads();
-  return bin;
+  if (in_bin) *in_bin = S.sel[2];
+  return S.sel[0];
+}
+
+// Zero the first nbins words of a histogram (nbins a multiple of 4, the array 16-byte aligned).
+__device__ __forceinline__ void clear_bins(uint32_t* h, int nbins) {
+  for (int i = threadIdx.x; i < nbins / 4; i += blockDim.x)
+    reinterpret_cast<uint4*>(h)[i] = make_uint4(0u, 0u, 0u, 0u);
 }
 
 __device__ __forceinline__ void topk_row(const float* __restrict__ src, int n, int topk,
@@ -479,7 +528,7 @@ __device__ __forceinline__ void topk_row(const float* __restrict__ src, int n, i
   if (hist1) {
     for (int i = tid; i < kTopkBins; i += kTopkThreads) S.hist[i] = hist1[i];
   } else {
-    for (int i = tid; i < kTopkBins; i += kTopkThreads) S.hist[i] = 0;
+    clear_bins(S.hist, kTopkBins);
     __syncthreads();
     for (int base = 0; base < n; base += kTopkThreads) {
       const int i = base + tid;
@@ -493,28 +542,28 @@ __device__ __forceinline__ void topk_row(const float* __restrict__ src, int n, i
   }
   __syncthreads();
   int above;
-  const uint32_t b1 = static_cast<uint32_t>(topk_find_bin(S, kTopkBins, need, &above));
+  const uint32_t b1 = static_cast<uint32_t>(topk_find_bin(S, S.hist, kTopkBins, need, &above));
   need -= above;
   // ---- digit 2: bits [19:8] among keys in bin b1 ----
-  for (int i = tid; i < kTopkBins; i += kTopkThreads) S.hist[i] = 0;
+  clear_bins(S.hist, kTopkBins);
   __syncthreads();
   for (int i = tid; i < n; i += kTopkThreads) {
     const uint32_t key = float_key(src[i]);
     if ((key >> 20) == b1) atomicAdd(&S.hist[(key >> 8) & 0xfffu], 1u);
   }
   __syncthreads();
-  const uint32_t b2 = static_cast<uint32_t>(topk_find_bin(S, kTopkBins, need, &above));
+  const uint32_t b2 = static_cast<uint32_t>(topk_find_bin(S, S.hist, kTopkBins, need, &above));
   need -= above;
   // ---- digit 3: bits [7:0] ----
   const uint32_t pre = (b1 << 12) | b2;
-  for (int i = tid; i < 256; i += kTopkThreads) S.hist[i] = 0;
+  clear_bins(S.hist, 256);
   __syncthreads();
   for (int i = tid; i < n; i += kTopkThreads) {
     const uint32_t key = float_key(src[i]);
     if ((key >> 8) == pre) atomicAdd(&S.hist[key & 0xffu], 1u);
   }
   __syncthreads();
-  const uint32_t b3 = static_cast<uint32_t>(topk_find_bin(S, 256, need, &above));
+  const uint32_t b3 = static_cast<uint32_t>(topk_find_bin(S, S.hist, 256, need, &above));
   need -= above;
   const uint32_t T = (pre << 8) | b3;   // the k-th largest key
   const int need_eq = need;             // keys equal to T to take, lowest indices first
@@ -597,7 +646,7 @@ __device__ __forceinline__ int hist_threshold_bin(const uint32_t* __restrict__ h
 #pragma unroll
   for (int j = 0; j < kCandBins; ++j) local += static_cast<int>(v[j]);
   int tot;
-  int running = block_excl_scan(local, sh, &tot);   // keys in bins above this thread's range
+  int running = block_excl_scan_1bar(local, sh, &tot);   // keys in bins above this thread's range
 #pragma unroll
   for (int j = kCandBins - 1; j >= 0; --j) {
     const int c = static_cast<int>(v[j]);
@@ -612,8 +661,7 @@ __device__ __forceinline__ int hist_threshold_bin(const uint32_t* __restrict__ h
   const int bin = sh[36];
   *above_out = sh[37];
   *in_bin_out = sh[38];
-  __syncthreads();
-  return bin;
+  return bin;   // sh[36..38] is not written again in this CTA
 }
 
 // Each CTA covers `per` (a multiple of 4) scores of one row in passes of 64 scores a thread
@@ -669,8 +717,11 @@ __global__ void __launch_bounds__(kCandThreads, 1) k_topk_collect(
       if (i < e && (float_key(x[j]) >> 20) >= b1) take |= 1ull << j;
     }
     int tot;
-    const int ex = block_excl_scan(__popcll(take), sh, &tot);
-    if (tot == 0) continue;   // uniform: tot is the block total
+    const int ex = block_excl_scan_1bar(__popcll(take), sh, &tot);
+    if (tot == 0) {            // uniform: tot is the block total
+      __syncthreads();         // the scan's totals are read before the next pass rewrites them
+      continue;
+    }
     if (threadIdx.x == 0) s_base = atomicAdd(cand_cnt + r, tot);
     __syncthreads();
     int slot = s_base + ex;
@@ -698,7 +749,8 @@ __device__ __forceinline__ void topk_select_candidates(TopkShared& S, const uint
                                                        int32_t* __restrict__ out) {
   const int tid = threadIdx.x;
   int above;
-  for (int i = tid; i < kTopkBins; i += blockDim.x) S.hist[i] = 0;
+  clear_bins(S.hist, kTopkBins);
+  clear_bins(S.hist3, 256);
   for (int i = tid; i < nwords; i += blockDim.x) {
     sel[i] = 0;
     eqb[i] = 0;
@@ -709,17 +761,15 @@ __device__ __forceinline__ void topk_select_candidates(TopkShared& S, const uint
     if ((key >> 20) == b1) atomicAdd(&S.hist[(key >> 8) & 0xfffu], 1u);
   }
   __syncthreads();
-  const uint32_t b2 = static_cast<uint32_t>(topk_find_bin(S, kTopkBins, need, &above));
+  const uint32_t b2 = static_cast<uint32_t>(topk_find_bin(S, S.hist, kTopkBins, need, &above));
   need -= above;
   const uint32_t pre = (b1 << 12) | b2;
-  for (int i = tid; i < 256; i += blockDim.x) S.hist[i] = 0;
-  __syncthreads();
   for (int i = tid; i < C; i += blockDim.x) {
     const uint32_t key = static_cast<uint32_t>(c[i] >> 32);
-    if ((key >> 8) == pre) atomicAdd(&S.hist[key & 0xffu], 1u);
+    if ((key >> 8) == pre) atomicAdd(&S.hist3[key & 0xffu], 1u);
   }
   __syncthreads();
-  const uint32_t b3 = static_cast<uint32_t>(topk_find_bin(S, 256, need, &above));
+  const uint32_t b3 = static_cast<uint32_t>(topk_find_bin(S, S.hist3, 256, need, &above));
   need -= above;
   const uint32_t T = (pre << 8) | b3;
   const int need_eq = need;
@@ -743,7 +793,7 @@ __device__ __forceinline__ void topk_select_candidates(TopkShared& S, const uint
       l_eq += __popc(eqb[w]);
     }
     int tot;
-    const int ex = block_excl_scan(l_eq * 2048 + l_gt, S.sh, &tot);
+    const int ex = block_excl_scan_1bar(l_eq * 2048 + l_gt, S.sh, &tot);
     const int eq_before = ex >> 11, gt_before = ex & 2047;
     int take = min(max(need_eq - eq_before, 0), l_eq);
     int pos = gt_before + min(eq_before, need_eq);
@@ -868,7 +918,7 @@ __global__ void __launch_bounds__(kTopkThreads, 4) k_topk(const float* __restric
     }
     const float* src = scores + r * ld;
     // ---- pass 1: first-digit histogram ----
-    for (int i = tid; i < kTopkBins; i += blockDim.x) S.hist[i] = 0;
+    clear_bins(S.hist, kTopkBins);
     if (tid == 0) s_cc = 0;
     __syncthreads();
     for (int base = 0; base < n; base += 4 * kTopkThreads) {
@@ -888,10 +938,8 @@ __global__ void __launch_bounds__(kTopkThreads, 4) k_topk(const float* __restric
         if (i0 + q < n) atomicAdd(&S.hist[float_key(x[q]) >> 20], 1u);
     }
     __syncthreads();
-    int above;
-    const uint32_t b1 = static_cast<uint32_t>(topk_find_bin(S, kTopkBins, topk, &above));
-    const int in_b1 = static_cast<int>(S.hist[b1]);
-    __syncthreads();   // every thread has read the histogram before it is rewritten
+    int above, in_b1;
+    const uint32_t b1 = static_cast<uint32_t>(topk_find_bin(S, S.hist, kTopkBins, topk, &above, &in_b1));
     if (above + in_b1 > cap) {
       topk_row(src, n, topk, nullptr, out, S);
       if (tid == 0) cnt[r] = topk;
@@ -1156,13 +1204,13 @@ __global__ void __launch_bounds__(kTopkThreads) k_merge_candidates(
   for (int j = K + tid; j < topk; j += blockDim.x) out[j] = -1;
   if (tid == 0) cnt[b] = K;
   if (K == 0) return;   // uniform
-  for (int i = tid; i < kTopkBins; i += blockDim.x) S.hist[i] = 0;
+  clear_bins(S.hist, kTopkBins);
   __syncthreads();
   for (int i = tid; i < C; i += blockDim.x)
     atomicAdd(&S.hist[static_cast<uint32_t>(c[i] >> 32) >> 20], 1u);
   __syncthreads();
   int above;
-  const uint32_t b1 = static_cast<uint32_t>(topk_find_bin(S, kTopkBins, K, &above));
+  const uint32_t b1 = static_cast<uint32_t>(topk_find_bin(S, S.hist, kTopkBins, K, &above));
   topk_select_candidates(S, c, C, b1, K - above, sel, eqb, nwords, K, out);
 }
 

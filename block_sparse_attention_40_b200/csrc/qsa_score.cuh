@@ -7,9 +7,10 @@
 // heads = 256 (prefill) or 1 token x 16 heads (decode) (B operand, loaded once per CTA),
 // K = 64.  The fp32 accumulator lives in TMEM (two buffers, so the epilogue of tile i
 // overlaps the MMA of tile i+1).  Epilogue: each thread owns one block row, reads its
-// 16 heads per token from TMEM, applies ReLU, weights by w and sums in fp32 (even and odd
-// heads as two partial sums), and writes the score if the block is a candidate of that token
-// (b < floor(pos/4)).
+// 16 heads per token from TMEM (prefill: four tokens, read as two pairs so that the second
+// read overlaps the sums of the first), applies ReLU, weights by w and sums in fp32 (even and
+// odd heads as two partial sums), and writes the score if the block is a candidate of that
+// token (b < floor(pos/4)).
 //
 // Warp roles: warp 0 issues TMA, warp 1 allocates TMEM and issues MMAs (one thread),
 // the remaining warps run the epilogue.
@@ -324,22 +325,35 @@ __global__ void __launch_bounds__(ScoreCfg<NTOK>::kThreads, ScoreCfg<NTOK>::kCta
       tc_fence_after();
       const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + a * C::kAccCols +
                              tok_base * kIdxHeads;
-      uint32_t acc[kTokPerWarp * kIdxHeads];
-      if constexpr (NTOK == 16) {
-#pragma unroll
-        for (int c = 0; c < kTokPerWarp / 2; ++c) tmem_ld32(tbase + 32 * c, acc + 32 * c);
-      } else {
-        tmem_ld16(tbase, acc);
-      }
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[a]);
-      const int blk = 128 * (wk.mt0 + i) + quarter * 32 + lane;
       float sc[kTokPerWarp];
-#pragma unroll
-      for (int j = 0; j < kTokPerWarp; ++j)
-        sc[j] = head_weighted_relu_sum(acc + j * kIdxHeads, sW + (tok_base + j) * kIdxHeads);
+      if constexpr (NTOK == 16) {
+        // two TMEM reads of two tokens each: the second is in flight while the first pair is
+        // summed, and the accumulator is released once both have landed
+        static_assert(kTokPerWarp == 4, "two pairs of tokens per warp");
+        uint32_t acc0[32], acc1[32];
+        tmem_ld32(tbase, acc0);
+        tmem_wait_ld();
+        reg_fence32(acc0);
+        tmem_ld32(tbase + 32, acc1);
+        sc[0] = head_weighted_relu_sum(acc0, sW + tok_base * kIdxHeads);
+        sc[1] = head_weighted_relu_sum(acc0 + kIdxHeads, sW + (tok_base + 1) * kIdxHeads);
+        tmem_wait_ld();
+        reg_fence32(acc1);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[a]);
+        sc[2] = head_weighted_relu_sum(acc1, sW + (tok_base + 2) * kIdxHeads);
+        sc[3] = head_weighted_relu_sum(acc1 + kIdxHeads, sW + (tok_base + 3) * kIdxHeads);
+      } else {
+        uint32_t acc[kIdxHeads];
+        tmem_ld16(tbase, acc);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[a]);
+        sc[0] = head_weighted_relu_sum(acc, sW + tok_base * kIdxHeads);
+      }
+      const int blk = 128 * (wk.mt0 + i) + quarter * 32 + lane;
 #pragma unroll
       for (int j = 0; j < kTokPerWarp; ++j) {
         const int tok = tok_base + j;
