@@ -355,6 +355,7 @@ def run_qsa(args, rank, world, local):
     if do_decode:
         errs.append(dec.device_error())
     assert all(e == ("QSA_OK", 0) for e in errs), errs
+    union = union_stats(idx, args.prefill_len, args.rows_per_tile or 10) if do_prefill else None
 
     # ---------------- e2e through host buffers ----------------
     e2e = {}
@@ -408,11 +409,35 @@ def run_qsa(args, rank, world, local):
 
     res = dict(sel_ms=sel_ms, att_ms=att_ms, dec_ms=dec_ms, clocks=clk, launches=launches,
                peaks=peaks, peak_src=peak_src, e2e=e2e, do_prefill=do_prefill,
-               do_decode=do_decode)
+               do_decode=do_decode, union=union)
     if do_decode:
         res["dec_bytes"] = sum(decode_bytes_per_seq(L + 1) for L in spec.context)
         res["dec_timing"] = "cuda graph replay of append + decode" if dec_graph is not None else "eager launches"
     return res
+
+
+def union_stats(idx, T, R):
+    """The prefill attention's union work, counted after the timed region from the selections
+    the step returned (one sequence of T tokens): each R-token tile attends the union of its
+    tokens' selected blocks and own blocks, in 32-block chunks of 128 keys for each KV head;
+    a chunk is 128 rows x 128 keys x 128 dims x 2 flops for QK^T and again for PV."""
+    import torch
+    k = idx.shape[1]
+    own = (torch.arange(T, device=idx.device, dtype=torch.int32) // 4)[:, None]
+    x = torch.cat([idx[:T], own], dim=1)
+    tiles = (T + R - 1) // R
+    if tiles * R > T:
+        x = torch.cat([x, torch.full((tiles * R - T, k + 1), -1, dtype=x.dtype,
+                                     device=x.device)])
+    x, _ = torch.sort(x.view(tiles, R * (k + 1)), dim=1)
+    first = torch.ones_like(x, dtype=torch.bool)
+    first[:, 1:] = x[:, 1:] != x[:, :-1]
+    u = ((x >= 0) & first).sum(dim=1)
+    chunks = int(((u + 31) // 32).sum().item()) * 2   # both KV heads
+    union_flops = chunks * 128 * 128 * 128 * 2 * 2
+    return {"rows_per_tile": R, "tiles": tiles, "union_blocks_per_tile": float(u.float().mean()),
+            "chunks": chunks, "union_tflop": union_flops / 1e12,
+            "useful_fraction": prefill_attention_flops(T) / union_flops}
 
 
 # ------------------------------------------------------------------------------------
@@ -704,7 +729,9 @@ def main():
                            "frac_of_bf16_peak_end_to_end":
                                attn_flops / (pre_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
                            "indexer_tflop": idx_flops / 1e12,
-                           "select_tflops_indexer_only": idx_flops / (r["sel_ms"] / K / 1e3) / 1e12}
+                           "select_tflops_indexer_only": idx_flops / (r["sel_ms"] / K / 1e3) / 1e12,
+                           "union": dict(r["union"], tensor_floor_ms=r["union"]["union_tflop"]
+                                         / peaks["bf16_tflops"] * 1e3)}
     if r["do_decode"]:
         dms = r["dec_ms"] / K
         gbs = r["dec_bytes"] / (dms / 1e3) / 1e9

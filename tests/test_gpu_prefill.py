@@ -1,4 +1,6 @@
 """GPU parity of QSA prefill (steps a1-a4) against the oracle."""
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -40,6 +42,25 @@ def test_short_sequences_and_dense_rows():
     p = W.custom_prefill([1, 2, 3, 4, 5, 9, 31, 64], topk=512, kind="normal", seed=5)
     idx, cnt, out = _run(p)
     prefill_oracle_check(p, idx, cnt, out, np.arange(int(p.cu_seqlens[-1])))
+
+
+@pytest.mark.parametrize("case", ["spread", "far_below", "far_above"])
+def test_attention_logits_far_from_zero(case):
+    # The attention logits q.k/sqrt(128) (log2 units) spread over hundreds of units within a
+    # row (q and k times 16, exact in bf16), or all lie about 260 units below or above zero
+    # (q = -4 or +4 in every dim, k shifted by +4): the softmax's running reference must move
+    # far within a row, and an exponent relative to a stale one would underflow or overflow.
+    # The selection comes from the indexer inputs, which stay as drawn.
+    p = W.custom_prefill([700, 333], topk=16, kind="normal", seed=11)
+    if case == "spread":
+        q, k = p.q.float() * 16, p.k.float() * 16
+    else:
+        q = torch.full_like(p.q, -4.0 if case == "far_below" else 4.0, dtype=torch.float32)
+        k = p.k.float() + 4
+    p = dataclasses.replace(p, q=q.bfloat16(), k=k.bfloat16())
+    idx, cnt, out = _run(p)
+    assert torch.isfinite(out.float()).all()
+    prefill_oracle_check(p, idx, cnt, out, np.arange(1033))
 
 
 def test_budget_one_and_chunked_scores():
