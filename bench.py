@@ -440,6 +440,55 @@ def union_stats(idx, T, R):
             "useful_fraction": prefill_attention_flops(T) / union_flops}
 
 
+GDN_LENGTHS, GDN_HEADS = [8192] * 8, 16
+
+
+def run_gdn(args, rank, world, local):
+    """The Gated DeltaNet layer (three of every four token-mixing layers around QSA) over 8
+    sequences of 8,192 tokens with 16 heads of 128, timed on its own after the rest.  Its
+    inputs (805 MB of q, k, v) exceed L2, so no flush is needed between launches."""
+    import torch
+    import block_sparse_attention_40_b200 as qsa
+    from block_sparse_attention_40_b200 import binding as B
+    from block_sparse_attention_40_b200 import workloads as W
+
+    dev = torch.device(f"cuda:{local}")
+    stream = torch.cuda.current_stream(dev)
+    w = W.gated_deltanet(GDN_LENGTHS, GDN_HEADS, seed=11 + rank, device=dev)
+    d_cu = w.cu_seqlens.to(dev)
+    out = torch.empty_like(w.q)
+    K = args.steps
+    clocks = ClockSampler(local)
+    clocks.start()
+    launches0 = B.launch_count()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    for i in range(args.warmup + K):
+        e = ev[i - args.warmup] if i >= args.warmup else None
+        if e:
+            e[0].record(stream)
+        qsa.gated_deltanet(w.q, w.k, w.v, w.log_alpha, w.beta, w.cu_seqlens, out=out,
+                           d_cu_seqlens=d_cu)
+        if e:
+            e[1].record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev) / K, world, dev)
+    T = sum(GDN_LENGTHS)
+    # the recurrence per token and head: S k, the rank-1 write and S q, 128 x 128 each
+    flops = 6 * 128 * 128 * T * GDN_HEADS
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    mhz = clk.get("sm_max_mhz") or 1965.0
+    peak = sms * 128 * 2 * mhz * 1e6 / 1e12   # fp32 FMA lanes per SM x 2 flops x clock
+    ach = flops / (ms / 1e3) / 1e12
+    return {"workload": f"{len(GDN_LENGTHS)} x {GDN_LENGTHS[0]} tokens, {GDN_HEADS} heads of 128",
+            "ms": ms, "tokens_per_s": world * T / (ms / 1e3),
+            "roofline": {"kernel": "k_gated_deltanet (fp32, chunks of 64 tokens)", "bound": "alu",
+                         "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+                         "peak_source": f"{sms} SMs x 128 fp32 FMA lanes x 2 x {mhz:.0f} MHz",
+                         "algorithmic": f"{flops / 1e12:.4f} TFLOP of the recurrence per launch"},
+            "clocks": clk, "gpu_launches": B.launch_count() - launches0}
+
+
 # ------------------------------------------------------------------------------------
 def ragged_attention_flops(lengths, k=TOPK):
     return sum(prefill_attention_flops(L, k) for L in lengths)
@@ -673,7 +722,8 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["qsa", "reference"], default="qsa")
-    ap.add_argument("--workload", choices=["both", "prefill", "decode"], default="both")
+    ap.add_argument("--workload", choices=["both", "prefill", "decode", "gdn"], default="both",
+                    help="gdn: only the Gated DeltaNet layer (a line of its own)")
     ap.add_argument("--rows-per-tile", type=int, default=0)
     ap.add_argument("--chunk-rows", type=int, default=0)
     ap.add_argument("--decode-splits", type=int, default=0)
@@ -688,6 +738,8 @@ def main():
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="time the decode step as eager launches instead of a CUDA graph replay")
     ap.add_argument("--no-cpu-baseline", dest="cpu", action="store_false")
+    ap.add_argument("--no-gdn", dest="gdn", action="store_false",
+                    help="skip the Gated DeltaNet layer timed after the rest")
     ap.add_argument("--no-mixed", dest="mixed", action="store_false",
                     help="skip the mixed ragged workload (8-sequence varlen prefill and the "
                          "1M-context decode) that follows the headline parts")
@@ -698,12 +750,30 @@ def main():
     if args.impl == "reference":
         run_reference(args, rank, world)
         return
+    if args.workload == "gdn":
+        gdn = run_gdn(args, rank, world, local)
+        if rank == 0:
+            print(json.dumps({
+                "metric": "Gated DeltaNet layer tokens/s", "value": gdn["tokens_per_s"],
+                "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": gdn["ms"], "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": {"workload": gdn["workload"], "l2": "inputs larger than L2",
+                           "parallelism": f"replicas x{world}"},
+                "roofline": gdn["roofline"], "clocks": gdn["clocks"],
+                "gpu_launches": gdn["gpu_launches"]}), flush=True)
+        return
     r = run_qsa(args, rank, world, local)
     mixed = None
     if args.mixed and args.workload == "both":
         import torch
         torch.cuda.empty_cache()
         mixed = run_mixed(args, rank, world, local)
+    gdn = None
+    if args.gdn and args.workload == "both":
+        import torch
+        torch.cuda.empty_cache()
+        gdn = run_gdn(args, rank, world, local)
     if rank != 0:
         return
     K = args.steps
@@ -764,6 +834,9 @@ def main():
     if mixed is not None:
         # the mixed ragged workload, timed separately after the headline step
         line["mixed_ragged"] = mixed
+    if gdn is not None:
+        # the Gated DeltaNet layer, timed separately after the rest
+        line["gated_deltanet"] = gdn
     if args.cpu and world == 1:
         line["cpu_baseline"] = cpu_baseline()
     print(json.dumps(line), flush=True)

@@ -5,4 +5,5 @@ The kernels and the C ABI live in ``csrc/`` and build into ``lib/libqsa.so`` (de
 ``workloads`` draws the seeded synthetic inputs.
 """
 from .binding import (KVCache, PagedKVCache, Decoder, Prefill, QSAError, compress, index_scores,  # noqa: F401
-                      last_device_error, load, prefill, prefill_select, topk, version)
+                      gated_deltanet, last_device_error, load, prefill, prefill_select, topk,
+                      version)

@@ -33,7 +33,7 @@ EXPORTS = ("qsa_status_string", "qsa_version", "qsa_launch_count", "qsa_workspac
            "qsa_decode_noalloc", "qsa_noalloc_last_device_error", "qsa_append_kv_paged",
            "qsa_decode_paged_workspace_size", "qsa_decode_paged",
            "qsa_decode_shard_workspace_size", "qsa_decode_shard_select", "qsa_merge_candidates",
-           "qsa_decode_shard_attend", "qsa_combine_partials")
+           "qsa_decode_shard_attend", "qsa_combine_partials", "qsa_gated_deltanet")
 
 
 class QSAError(RuntimeError):
@@ -104,6 +104,7 @@ def load(build_if_needed: bool = True):
             "qsa_merge_candidates": ([P, P, P, I32, I32, I32, I32, P, P, P, SZ, P], st),
             "qsa_decode_shard_attend": ([P, P, I32, P, P, P, P, P, P, P, SZ, Params, P], st),
             "qsa_combine_partials": ([P, P, P, I32, I32, P, P], st),
+            "qsa_gated_deltanet": ([P, P, P, P, P, P, P, I32, I32, P, P, P], st),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -604,3 +605,33 @@ def combine_partials(part_o, part_m, part_l, out=None):
     _check("qsa_combine_partials", load().qsa_combine_partials(
         _ptr(part_o), _ptr(part_m), _ptr(part_l), R, B, _ptr(out), _stream(part_o.device)))
     return out
+
+
+def gated_deltanet(q, k, v, log_alpha, beta, cu_seqlens, out=None, with_state=False,
+                   d_cu_seqlens=None):
+    """The Gated DeltaNet layer over packed sequences: q, k, v bf16 [T, H, 128], log_alpha and
+    beta fp32 [T, H] -> out bf16 [T, H, 128] (and the final states fp32 [S, H, 128, 128]).
+    d_cu_seqlens: a device copy of cu_seqlens (host) to reuse instead of copying it."""
+    dev = q.device
+    if d_cu_seqlens is not None:
+        h, d = torch.as_tensor(cu_seqlens, dtype=torch.int32).contiguous(), d_cu_seqlens
+    else:
+        h, d = _cu_pair(cu_seqlens, dev)
+    T = int(h[-1])
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, torch.bfloat16, (q.shape[1], 128), 3)
+        if t.shape[0] != T:
+            raise ValueError(f"{name}: {t.shape[0]} tokens, cu_seqlens says {T}")
+    H = q.shape[1]
+    for name, t in (("log_alpha", log_alpha), ("beta", beta)):
+        _need(t, name, torch.float32, (H,), 2)
+        if t.shape[0] != T:
+            raise ValueError(f"{name}: {t.shape[0]} tokens, cu_seqlens says {T}")
+    if out is None:
+        out = torch.empty_like(q)
+    S = h.numel() - 1
+    state = torch.empty((S, H, 128, 128), dtype=torch.float32, device=dev) if with_state else None
+    _check("qsa_gated_deltanet", load().qsa_gated_deltanet(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(d),
+        ctypes.c_void_p(h.data_ptr()), S, H, _ptr(out), _ptr(state), _stream(dev)))
+    return (out, state) if with_state else out

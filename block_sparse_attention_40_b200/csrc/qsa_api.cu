@@ -11,6 +11,7 @@
 #include "../../include/qsa.h"
 #include "qsa_attn.cuh"
 #include "qsa_common.cuh"
+#include "qsa_gdn.cuh"
 #include "qsa_misc.cuh"
 #include "qsa_score.cuh"
 
@@ -1146,4 +1147,35 @@ extern "C" qsa_status qsa_noalloc_last_device_error(qsa_stream_t stream, uint32_
   if (site) *site = h[1];
   if (h[0] == 0) return QSA_OK;
   return h[0] == kErrTimeout ? QSA_ERR_TIMEOUT : QSA_ERR_DEVICE;
+}
+
+// ---- the Gated DeltaNet layer ------------------------------------------------------------
+extern "C" qsa_status qsa_gated_deltanet(const void* q, const void* k, const void* v,
+                                         const float* log_alpha, const float* beta,
+                                         const int32_t* d_cu_seqlens, const int32_t* h_cu_seqlens,
+                                         int32_t num_seqs, int32_t heads, void* out,
+                                         float* final_state, qsa_stream_t stream) {
+  if (!q || !k || !v || !log_alpha || !beta || !d_cu_seqlens || !h_cu_seqlens || !out)
+    return QSA_ERR_INVALID_ARG;
+  if (num_seqs < 1 || num_seqs > 65535 || heads < 1 || heads > 256) return QSA_ERR_INVALID_ARG;
+  if (h_cu_seqlens[0] != 0) return QSA_ERR_INVALID_ARG;
+  for (int32_t i = 0; i < num_seqs; ++i)
+    if (h_cu_seqlens[i + 1] < h_cu_seqlens[i]) return QSA_ERR_INVALID_ARG;
+  for (const void* p : {q, k, v, static_cast<const void*>(out)})
+    if (!aligned16(p)) return QSA_ERR_ALIGNMENT;
+  if (!set_smem(k_gated_deltanet, kGdnSmemBytes)) return QSA_ERR_CUDA;
+  GdnArgs a{};
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k = static_cast<const __nv_bfloat16*>(k);
+  a.v = static_cast<const __nv_bfloat16*>(v);
+  a.log_alpha = log_alpha;
+  a.beta = beta;
+  a.cu = d_cu_seqlens;
+  a.heads = heads;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.final_state = final_state;
+  k_gated_deltanet<<<dim3(heads, num_seqs), kGdnThreads, kGdnSmemBytes,
+                     reinterpret_cast<cudaStream_t>(stream)>>>(a);
+  QSA_CHECK_LAUNCH();
+  return QSA_OK;
 }

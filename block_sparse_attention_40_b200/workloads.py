@@ -248,3 +248,45 @@ def bits(t: torch.Tensor):
     """Raw bf16 bit patterns of a tensor as a numpy uint16 array (CPU copy)."""
     assert t.dtype == torch.bfloat16
     return t.detach().contiguous().cpu().view(torch.int16).numpy().view("uint16")
+
+
+# ---- the Gated DeltaNet layer ------------------------------------------------------------
+@dataclasses.dataclass
+class GatedDeltaNet:
+    q: torch.Tensor          # [T, H, 128] bf16, each row of unit L2 norm (before bf16 rounding)
+    k: torch.Tensor          # [T, H, 128] bf16, likewise
+    v: torch.Tensor          # [T, H, 128] bf16, N(0,1)
+    log_alpha: torch.Tensor  # [T, H] fp32: log of a gate drawn uniformly in `gate`
+    beta: torch.Tensor       # [T, H] fp32, U(0,1)
+    cu_seqlens: torch.Tensor  # [num_seqs+1] int32 (CPU)
+
+    def to(self, device) -> "GatedDeltaNet":
+        kw = {f.name: getattr(self, f.name) for f in dataclasses.fields(self)}
+        for n in ("q", "k", "v", "log_alpha", "beta"):
+            kw[n] = kw[n].to(device)
+        return GatedDeltaNet(**kw)
+
+
+def gated_deltanet(lengths, heads, seed=0, gate=(0.9, 1.0), reset_every=0, device="cpu"):
+    """Seeded inputs of the Gated DeltaNet layer for packed sequences of the given lengths.
+    q and k are unit-norm rows (the layer takes them as given; normalised keys keep the
+    delta rule's state bounded), gates alpha ~ U(gate), and with reset_every > 0 every
+    reset_every-th token has alpha = 0 (log_alpha = -inf)."""
+    g = torch.Generator().manual_seed(5000 + seed)
+    T = int(sum(lengths))
+    shape = (T, heads, HEAD_DIM)
+
+    def unit_rows():
+        x = torch.randn(shape, generator=g)
+        return (x / x.norm(dim=-1, keepdim=True).clamp_min(1e-6)).to(torch.bfloat16)
+
+    q, k = unit_rows(), unit_rows()
+    v = torch.randn(shape, generator=g).to(torch.bfloat16)
+    lo, hi = gate
+    log_alpha = torch.log(lo + (hi - lo) * torch.rand((T, heads), generator=g))
+    if reset_every > 0:
+        log_alpha[::reset_every] = float("-inf")
+    beta = torch.rand((T, heads), generator=g)
+    cu = torch.tensor([0] + torch.tensor([int(x) for x in lengths]).cumsum(0).tolist(),
+                      dtype=torch.int32)
+    return GatedDeltaNet(q, k, v, log_alpha, beta, cu).to(device)

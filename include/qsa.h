@@ -376,6 +376,31 @@ QSA_API qsa_status qsa_decode_paged(const void *q, const qsa_paged_cache *cache,
                                     void *workspace, size_t ws_bytes, qsa_params params,
                                     qsa_stream_t stream);
 
+/* ---------------------------------------------------------------------------------- */
+/* The Gated DeltaNet layer, prefill over packed variable-length sequences ("Long context
+ * became an architecture problem", "Linear attention carries the stream; sparse attention
+ * retrieves detail": Gated DeltaNet, a gated linear recurrence over a compact state, carries
+ * three of every four token-mixing layers; the pages' table of its parameters is lost, so
+ * the update is the published gated delta rule).  Per sequence and head, the state S
+ * (128 x 128, fp32) starts at zero, and token t updates it and reads it out:
+ *     S_t = alpha_t S_{t-1} + beta_t (v_t - alpha_t S_{t-1} k_t) k_t^T,    o_t = S_t q_t
+ * with alpha_t = exp(log_alpha_t).  q and k are used as given (any normalisation or scaling
+ * happens before the call); log_alpha below -87 counts as -87 (a full reset, to fp32 range).
+ *   q, k, v      bf16 [T][heads][128], 16-byte aligned
+ *   log_alpha    fp32 [T][heads] (<= 0 keeps the state bounded), beta fp32 [T][heads]
+ *   d_cu_seqlens int32 [num_seqs+1] on the device, h_cu_seqlens the same on the host
+ *                (0 = cu[0] <= cu[1] <= ...; sequences may be empty)
+ *   out          bf16 [T][heads][128] output, 16-byte aligned (caller-owned)
+ *   final_state  fp32 [num_seqs][heads][128 (v)][128 (k)] output: S after each sequence's
+ *                last token, or NULL
+ * heads 1..256.  No workspace.  Errors: QSA_ERR_INVALID_ARG (null pointer, bad sizes or
+ * cu_seqlens), QSA_ERR_ALIGNMENT, QSA_ERR_CUDA (launch failure).  Asynchronous on stream. */
+QSA_API qsa_status qsa_gated_deltanet(const void *q, const void *k, const void *v,
+                                      const float *log_alpha, const float *beta,
+                                      const int32_t *d_cu_seqlens, const int32_t *h_cu_seqlens,
+                                      int32_t num_seqs, int32_t heads, void *out,
+                                      float *final_state, qsa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
