@@ -42,18 +42,18 @@ DEC_BATCH, DEC_CAP = 64, 262144
 # figure is reported only while the sources are unchanged; otherwise the roofline's
 # "traffic" is null until a new capture is taken.
 NCU_TRAFFIC = {
-    # 314,285,056 B read + 174,872,064 B written by one 32K-token prefill attention launch
+    # 312,913,920 B read + 175,029,248 B written by one 32K-token prefill attention launch
     # (profiles/k_sparse_attn_prefill_32k.md), per token; the attention's bytes (Q, O, the
     # gathered K/V tiles, the plan) grow with the tokens of the launch.
-    "prefill_attention": (489157120 / 32768,
-                          "f8b96856055c90939ba9d5a3cd0d78750e7cbe709c96d7c562f9745e2cc35c54",
+    "prefill_attention": (487943168 / 32768,
+                          "bbeeb2e7c056e7a6a039c1f3c45394ed7199c42e5dfda990eee1020e6c47f3ec",
                           "ncu dram__bytes_read.sum + dram__bytes_write.sum of one 32K-token "
                           "launch (profiles/k_sparse_attn_prefill_32k.md), scaled by tokens"),
     # The seven kernels of one 256K x 64 decode step, one ncu capture each (1 pass): reads
-    # 690,930,432 B, writes 6,806,784 B (profiles/decode_step_dram_decode256k_b64.md); per
+    # 690,877,440 B, writes 6,624,768 B (profiles/decode_step_dram_decode256k_b64.md); per
     # sequence of the batch.
-    "decode_step": (697737216 / 64,
-                    "c4a9bcabd65325ff2d9053c1713f493faa5e21cffd98b72f4345ff77196e98b5",
+    "decode_step": (697502208 / 64,
+                    "9cfeb5904dc5ca654888985d6cb15d446fbdba0980d58d3daf32f6f9c9dc8737",
                     "ncu dram__bytes_read.sum + dram__bytes_write.sum of the seven kernels of "
                     "one 256K x 64 decode step (profiles/decode_step_dram_decode256k_b64.md)"),
 }
@@ -63,7 +63,8 @@ NCU_TRAFFIC = {
 # of them changes.
 TRAFFIC_SOURCES = {
     "prefill_attention": ("qsa_attn.cuh", "qsa_common.cuh", "qsa_api.cu"),
-    "decode_step": None,   # the whole step: every source
+    "decode_step": ("qsa_api.cu", "qsa_attn.cuh", "qsa_common.cuh", "qsa_misc.cuh",
+                    "qsa_score.cuh"),   # the whole step
 }
 
 
