@@ -28,13 +28,16 @@ namespace qsa {
 constexpr int kGdnDim = 128;      // d_k = d_v
 constexpr int kGdnChunk = 64;
 constexpr int kGdnThreads = 512;
-constexpr int kGdnKStride = kGdnDim + 1;   // K rows padded: column reads across lanes hit distinct banks
+constexpr int kGdnKStride = kGdnDim + 4;   // K rows padded: 16-byte rows, 4-way at most on column stores
 constexpr float kGdnMinLogAlpha = -87.f;
 
+// Operands are laid out so that every product reads them as float4: K and Q also held
+// transposed (k-major, tokens contiguous), so a thread's four rows arrive in one broadcast.
 struct GdnSmem {
   float st[kGdnDim * kGdnDim];          // S^T: st[k][v]
-  float k[kGdnChunk * kGdnKStride];     // K rows (padded)
-  float q[kGdnChunk * kGdnDim];
+  float k[kGdnChunk * kGdnKStride];     // K rows (padded): k[t][d]
+  float kt[kGdnDim * kGdnChunk];        // K^T: kt[d][t]
+  float qt[kGdnDim * kGdnChunk];        // Q^T: qt[d][t]
   float v[kGdnChunk * kGdnDim];         // V, then V - diag(e^g) K S0^T, then U
   float a[kGdnChunk * kGdnChunk];       // A (strictly lower)
   float m[kGdnChunk * kGdnChunk];       // M (lower, diagonal included)
@@ -64,27 +67,41 @@ __device__ __forceinline__ float bf16_bits_to_float(uint32_t b) { return __uint_
 __device__ __forceinline__ void gdn_load_chunk(const GdnArgs& a, GdnSmem& S, int h, int64_t t0,
                                                int n) {
   const int tid = threadIdx.x;
-  // 64 rows x 128 dims = 1024 groups of 8 bf16 per matrix, two per thread
+  // q and k: lanes take consecutive tokens (so the transposed stores are conflict-free);
+  // v: lanes take consecutive 8-value groups of a row.  1024 groups of 8 bf16 per matrix.
   for (int e = tid; e < kGdnChunk * (kGdnDim / 8); e += kGdnThreads) {
-    const int t = e / (kGdnDim / 8), d0 = (e % (kGdnDim / 8)) * 8;
-    uint4 rq = make_uint4(0u, 0u, 0u, 0u), rk = rq, rv = rq;
+    const int t = e % kGdnChunk, d0 = (e / kGdnChunk) * 8;
+    uint4 rq = make_uint4(0u, 0u, 0u, 0u), rk = rq;
     if (t < n) {
       const int64_t off = ((t0 + t) * a.heads + h) * kGdnDim + d0;
       rq = *reinterpret_cast<const uint4*>(a.q + off);
       rk = *reinterpret_cast<const uint4*>(a.k + off);
-      rv = *reinterpret_cast<const uint4*>(a.v + off);
     }
-    const uint32_t wq[4] = {rq.x, rq.y, rq.z, rq.w}, wk[4] = {rk.x, rk.y, rk.z, rk.w},
-                   wv[4] = {rv.x, rv.y, rv.z, rv.w};
+    const uint32_t wq[4] = {rq.x, rq.y, rq.z, rq.w}, wk[4] = {rk.x, rk.y, rk.z, rk.w};
+    float kf[8];
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
-      S.q[t * kGdnDim + d0 + 2 * p] = bf16_bits_to_float(wq[p] & 0xffffu);
-      S.q[t * kGdnDim + d0 + 2 * p + 1] = bf16_bits_to_float(wq[p] >> 16);
-      S.k[t * kGdnKStride + d0 + 2 * p] = bf16_bits_to_float(wk[p] & 0xffffu);
-      S.k[t * kGdnKStride + d0 + 2 * p + 1] = bf16_bits_to_float(wk[p] >> 16);
-      S.v[t * kGdnDim + d0 + 2 * p] = bf16_bits_to_float(wv[p] & 0xffffu);
-      S.v[t * kGdnDim + d0 + 2 * p + 1] = bf16_bits_to_float(wv[p] >> 16);
+      S.qt[(d0 + 2 * p) * kGdnChunk + t] = bf16_bits_to_float(wq[p] & 0xffffu);
+      S.qt[(d0 + 2 * p + 1) * kGdnChunk + t] = bf16_bits_to_float(wq[p] >> 16);
+      kf[2 * p] = bf16_bits_to_float(wk[p] & 0xffffu);
+      kf[2 * p + 1] = bf16_bits_to_float(wk[p] >> 16);
     }
+#pragma unroll
+    for (int p = 0; p < 8; ++p) S.kt[(d0 + p) * kGdnChunk + t] = kf[p];
+    float4* kr = reinterpret_cast<float4*>(&S.k[t * kGdnKStride + d0]);
+    kr[0] = make_float4(kf[0], kf[1], kf[2], kf[3]);
+    kr[1] = make_float4(kf[4], kf[5], kf[6], kf[7]);
+  }
+  for (int e = tid; e < kGdnChunk * (kGdnDim / 8); e += kGdnThreads) {
+    const int t = e / (kGdnDim / 8), d0 = (e % (kGdnDim / 8)) * 8;
+    uint4 rv = make_uint4(0u, 0u, 0u, 0u);
+    if (t < n) rv = *reinterpret_cast<const uint4*>(a.v + ((t0 + t) * a.heads + h) * kGdnDim + d0);
+    const uint32_t wv[4] = {rv.x, rv.y, rv.z, rv.w};
+    float4* vr = reinterpret_cast<float4*>(&S.v[t * kGdnDim + d0]);
+    vr[0] = make_float4(bf16_bits_to_float(wv[0] & 0xffffu), bf16_bits_to_float(wv[0] >> 16),
+                        bf16_bits_to_float(wv[1] & 0xffffu), bf16_bits_to_float(wv[1] >> 16));
+    vr[1] = make_float4(bf16_bits_to_float(wv[2] & 0xffffu), bf16_bits_to_float(wv[2] >> 16),
+                        bf16_bits_to_float(wv[3] & 0xffffu), bf16_bits_to_float(wv[3] >> 16));
   }
   // gates: warp 0, two tokens a lane, an inclusive scan of the clamped log gates
   if (tid < 32) {
@@ -139,15 +156,16 @@ __global__ void __launch_bounds__(kGdnThreads, 1) k_gated_deltanet(GdnArgs a) {
 #pragma unroll 4
       for (int kk = 0; kk < kGdnDim; ++kk) {
         const float4 s4 = *reinterpret_cast<const float4*>(&S.st[kk * kGdnDim + 4 * lane]);
+        const float4 k4 = *reinterpret_cast<const float4*>(&S.kt[kk * kGdnChunk + 4 * warp]);
+        const float4 q4 = *reinterpret_cast<const float4*>(&S.qt[kk * kGdnChunk + 4 * warp]);
         const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+        const float kr[4] = {k4.x, k4.y, k4.z, k4.w}, qr[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-          const float kr = S.k[(4 * warp + r) * kGdnKStride + kk];
-          const float qr = S.q[(4 * warp + r) * kGdnDim + kk];
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            ak[r][c] = fmaf(kr, sv[c], ak[r][c]);
-            aq[r][c] = fmaf(qr, sv[c], aq[r][c]);
+            ak[r][c] = fmaf(kr[r], sv[c], ak[r][c]);
+            aq[r][c] = fmaf(qr[r], sv[c], aq[r][c]);
           }
         }
       }
@@ -173,16 +191,16 @@ __global__ void __launch_bounds__(kGdnThreads, 1) k_gated_deltanet(GdnArgs a) {
       for (int r = 0; r < 4; ++r) ka[r][0] = ka[r][1] = qa[r][0] = qa[r][1] = 0.f;
 #pragma unroll 4
       for (int kk = 0; kk < kGdnDim; ++kk) {
-        const float kj0 = S.k[(2 * lane) * kGdnKStride + kk];
-        const float kj1 = S.k[(2 * lane + 1) * kGdnKStride + kk];
+        const float2 kj = *reinterpret_cast<const float2*>(&S.kt[kk * kGdnChunk + 2 * lane]);
+        const float4 k4 = *reinterpret_cast<const float4*>(&S.kt[kk * kGdnChunk + 4 * warp]);
+        const float4 q4 = *reinterpret_cast<const float4*>(&S.qt[kk * kGdnChunk + 4 * warp]);
+        const float kr[4] = {k4.x, k4.y, k4.z, k4.w}, qr[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-          const float kr = S.k[(4 * warp + r) * kGdnKStride + kk];
-          const float qr = S.q[(4 * warp + r) * kGdnDim + kk];
-          ka[r][0] = fmaf(kr, kj0, ka[r][0]);
-          ka[r][1] = fmaf(kr, kj1, ka[r][1]);
-          qa[r][0] = fmaf(qr, kj0, qa[r][0]);
-          qa[r][1] = fmaf(qr, kj1, qa[r][1]);
+          ka[r][0] = fmaf(kr[r], kj.x, ka[r][0]);
+          ka[r][1] = fmaf(kr[r], kj.y, ka[r][1]);
+          qa[r][0] = fmaf(qr[r], kj.x, qa[r][0]);
+          qa[r][1] = fmaf(qr[r], kj.y, qa[r][1]);
         }
       }
 #pragma unroll
@@ -260,9 +278,11 @@ __global__ void __launch_bounds__(kGdnThreads, 1) k_gated_deltanet(GdnArgs a) {
         const float4* up = reinterpret_cast<const float4*>(&S.v[t * kGdnDim + 8 * vb]);
         const float4 x = up[0], y = up[1];
         const float uv[8] = {x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
+        const float4 k4 = *reinterpret_cast<const float4*>(&S.k[t * kGdnKStride + 4 * kb]);
+        const float kw[4] = {w * k4.x, w * k4.y, w * k4.z, w * k4.w};
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-          const float kr = w * S.k[t * kGdnKStride + 4 * kb + r];
+          const float kr = kw[r];
 #pragma unroll
           for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(kr, uv[c], acc[r][c]);
         }
