@@ -42,18 +42,18 @@ DEC_BATCH, DEC_CAP = 64, 262144
 # figure is reported only while the sources are unchanged; otherwise the roofline's
 # "traffic" is null until a new capture is taken.
 NCU_TRAFFIC = {
-    # 312,913,920 B read + 175,029,248 B written by one 32K-token prefill attention launch
+    # 313,151,232 B read + 174,985,728 B written by one 32K-token prefill attention launch
     # (profiles/k_sparse_attn_prefill_32k.md), per token; the attention's bytes (Q, O, the
     # gathered K/V tiles, the plan) grow with the tokens of the launch.
-    "prefill_attention": (487943168 / 32768,
-                          "bbeeb2e7c056e7a6a039c1f3c45394ed7199c42e5dfda990eee1020e6c47f3ec",
+    "prefill_attention": (488136960 / 32768,
+                          "dddb15f8abeac87cf6d17bf4cb9d3c5040e9da29c053e377eb7f9eac688ef064",
                           "ncu dram__bytes_read.sum + dram__bytes_write.sum of one 32K-token "
                           "launch (profiles/k_sparse_attn_prefill_32k.md), scaled by tokens"),
     # The seven kernels of one 256K x 64 decode step, one ncu capture each (1 pass): reads
-    # 690,877,440 B, writes 6,624,768 B (profiles/decode_step_dram_decode256k_b64.md); per
+    # 690,881,024 B, writes 6,595,328 B (profiles/decode_step_dram_decode256k_b64.md); per
     # sequence of the batch.
-    "decode_step": (697502208 / 64,
-                    "9cfeb5904dc5ca654888985d6cb15d446fbdba0980d58d3daf32f6f9c9dc8737",
+    "decode_step": (697476352 / 64,
+                    "fadf51d78a57630cac8be444066970114157d9a5107edaf43e92b098665b510b",
                     "ncu dram__bytes_read.sum + dram__bytes_write.sum of the seven kernels of "
                     "one 256K x 64 decode step (profiles/decode_step_dram_decode256k_b64.md)"),
 }
@@ -244,7 +244,8 @@ def run_qsa(args, rank, world, local):
         else:   # smaller case of the same drifting workload (profiling captures)
             p = W.custom_prefill([args.prefill_len], TOPK, kind="drift", device=dev,
                                  seed=1002 + rank)
-        ctx = qsa.Prefill(p.cu_seqlens, dev, TOPK, args.rows_per_tile, args.chunk_rows)
+        ctx = qsa.Prefill(p.cu_seqlens, dev, TOPK, args.rows_per_tile, args.chunk_rows,
+                          select_mode=args.select_mode)
         idx = torch.empty((args.prefill_len, TOPK), dtype=torch.int32, device=dev)
         cnt = torch.empty((args.prefill_len,), dtype=torch.int32, device=dev)
         out = torch.empty_like(p.q)
@@ -675,7 +676,7 @@ def workload_config(args, world, do_prefill, do_decode):
             "decode_context": "262140 + (i mod 4)", "topk_blocks": TOPK,
             "heads": "24q/2kv", "head_dim": 128, "indexer": "16x64",
             "l2": "flushed before each timed part (256 MB write, then 256 MB read)",
-            "parallelism": f"replicas x{world}"}
+            "parallelism": f"replicas x{world}", "select_mode": args.select_mode}
 
 
 def run_reference(args, rank, world):
@@ -739,6 +740,9 @@ def main():
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="time the decode step as eager launches instead of a CUDA graph replay")
     ap.add_argument("--no-cpu-baseline", dest="cpu", action="store_false")
+    ap.add_argument("--select-mode", type=int, default=0,
+                    help="prefill selection: 0 = default; 1 = the indexer finds each row's "
+                         "threshold bin (the fused index-score + select)")
     ap.add_argument("--no-gdn", dest="gdn", action="store_false",
                     help="skip the Gated DeltaNet layer timed after the rest")
     ap.add_argument("--no-mixed", dest="mixed", action="store_false",

@@ -45,7 +45,7 @@ class QSAError(RuntimeError):
 class Params(ctypes.Structure):
     _fields_ = [("topk_blocks", ctypes.c_int32), ("rows_per_tile", ctypes.c_int32),
                 ("decode_splits", ctypes.c_int32), ("score_chunk_rows", ctypes.c_int32),
-                ("debug_fault", ctypes.c_int32)]
+                ("debug_fault", ctypes.c_int32), ("select_mode", ctypes.c_int32)]
 
 
 class CacheDesc(ctypes.Structure):
@@ -157,9 +157,10 @@ def _cu_pair(cu_seqlens, device):
     return h, d
 
 
-def _params(topk, rows_per_tile=0, decode_splits=0, score_chunk_rows=0, debug_fault=0) -> Params:
+def _params(topk, rows_per_tile=0, decode_splits=0, score_chunk_rows=0, debug_fault=0,
+            select_mode=0) -> Params:
     return Params(int(topk), int(rows_per_tile), int(decode_splits), int(score_chunk_rows),
-                  int(debug_fault))
+                  int(debug_fault), int(select_mode))
 
 
 def new_workspace(nbytes: int, device) -> torch.Tensor:
@@ -190,11 +191,13 @@ def launch_count() -> int:
 
 
 # --------------------------------------------------------------------------------------
-def prefill_workspace_size(cu_seqlens_host, topk=512, rows_per_tile=0, score_chunk_rows=0) -> int:
+def prefill_workspace_size(cu_seqlens_host, topk=512, rows_per_tile=0, score_chunk_rows=0,
+                           select_mode=0) -> int:
     h = torch.as_tensor(cu_seqlens_host, dtype=torch.int32).contiguous()
     n = load().qsa_prefill_workspace_size(ctypes.c_void_p(h.data_ptr()),
                                           h.numel() - 1,
-                                          _params(topk, rows_per_tile, 0, score_chunk_rows))
+                                          _params(topk, rows_per_tile, 0, score_chunk_rows,
+                                                  0, select_mode))
     if n == 0:
         raise QSAError("qsa_prefill_workspace_size", 1)
     return int(n)
@@ -280,15 +283,16 @@ class Prefill:
     """Reusable prefill context: holds the device cu_seqlens and the workspace."""
 
     def __init__(self, cu_seqlens, device, topk=512, rows_per_tile=0, score_chunk_rows=0,
-                 debug_fault=0):
+                 debug_fault=0, select_mode=0):
         self.device = torch.device(device)
         self.h_cu, self.d_cu = _cu_pair(cu_seqlens, self.device)
         self.num_seqs = self.h_cu.numel() - 1
         self.T = int(self.h_cu[-1])
-        self.params = _params(topk, rows_per_tile, 0, score_chunk_rows, debug_fault)
+        self.params = _params(topk, rows_per_tile, 0, score_chunk_rows, debug_fault, select_mode)
         self.topk = int(topk)
         self.ws = new_workspace(prefill_workspace_size(self.h_cu, topk, rows_per_tile,
-                                                       score_chunk_rows), self.device)
+                                                       score_chunk_rows, select_mode),
+                                self.device)
         self.lib = load()
 
     def run(self, q, k, v, q_idx, k_idx, w, out=None):

@@ -100,10 +100,12 @@ struct PrefillGeom {
   int32_t topk = 512;
   int32_t chunk_rows = kDefaultScoreChunkRows;
   int32_t fault = 0;   // qsa_params.debug_fault
+  bool fused = false;  // qsa_params.select_mode 1 applies: the indexer finds each row's threshold bin
   PlanLayout pl;
   int32_t max_words = 1;
   // workspace offsets
-  size_t o_meta = 0, o_kbar = 0, o_nc = 0, o_scores = 0, o_idx = 0, o_cnt = 0, o_plan = 0, total = 0;
+  size_t o_meta = 0, o_kbar = 0, o_nc = 0, o_scores = 0, o_rinfo = 0, o_idx = 0, o_cnt = 0,
+         o_plan = 0, total = 0;
 };
 
 qsa_status prefill_geom(const int32_t* h_cu, int32_t num_seqs, const qsa_params& p,
@@ -111,6 +113,7 @@ qsa_status prefill_geom(const int32_t* h_cu, int32_t num_seqs, const qsa_params&
   if (!h_cu || num_seqs <= 0) return QSA_ERR_INVALID_ARG;
   if (p.topk_blocks < 1 || p.topk_blocks > QSA_MAX_TOPK) return QSA_ERR_INVALID_ARG;
   if (p.debug_fault != 0 && p.debug_fault != 1) return QSA_ERR_INVALID_ARG;
+  if (p.select_mode != 0 && p.select_mode != 1) return QSA_ERR_INVALID_ARG;
   if (h_cu[0] != 0) return QSA_ERR_INVALID_ARG;
   g->fault = p.debug_fault;
   g->R = p.rows_per_tile > 0 ? p.rows_per_tile : kDefaultRowsPerTile;
@@ -135,6 +138,8 @@ qsa_status prefill_geom(const int32_t* h_cu, int32_t num_seqs, const qsa_params&
   g->max_len = max_len;
   g->total_blocks = blocks;
   g->max_nc = (max_len - 1) / 4;
+  // the indexer's per-row histograms count in 16 bits: rows of fewer than 65,536 candidates
+  g->fused = p.select_mode == 1 && g->max_nc < 65536;
   g->ld = std::max<int64_t>(4, round_up(std::max(g->max_nc, 1), 4));
   g->score_tiles = static_cast<int32_t>(st);
   g->attn_tiles = static_cast<int32_t>(at);
@@ -146,6 +151,7 @@ qsa_status prefill_geom(const int32_t* h_cu, int32_t num_seqs, const qsa_params&
   g->o_nc = c.take(static_cast<size_t>(T) * 4);
   const int64_t rows = std::min<int64_t>(T, g->chunk_rows + 16);
   g->o_scores = c.take(static_cast<size_t>(rows) * g->ld * 4);
+  if (g->fused) g->o_rinfo = c.take(static_cast<size_t>(rows) * 4 * 4);   // threshold bin per row
   g->o_idx = c.take(static_cast<size_t>(T) * g->topk * 4);
   g->o_cnt = c.take(static_cast<size_t>(T) * 4);
   g->o_plan = c.take(static_cast<size_t>(g->attn_tiles) * g->pl.stride * 4);
@@ -225,15 +231,17 @@ qsa_status launch_compress(const void* k_idx, const SeqMeta* meta, int num_seqs,
 }
 
 // Top-k over `rows` score rows (one CTA per row, grid-strided).
+// rinfo: each row's threshold bin as the indexer found it (select_mode 1), or null.
 qsa_status launch_topk(const float* scores, int64_t ld, const int32_t* n_c, int64_t rows,
-                       int topk, int max_nc, int32_t* idx, int32_t* cnt, cudaStream_t s) {
+                       int topk, int max_nc, int32_t* idx, int32_t* cnt, cudaStream_t s,
+                       const int32_t* rinfo = nullptr) {
   if (rows <= 0) return QSA_OK;
   const int n_max = std::max(max_nc, 1);
   const int smem = kTopkSharedBytes + kTopkCandCap * 8 + 2 * ((n_max + 31) / 32) * 4;
   if (!set_smem(k_topk, smem)) return QSA_ERR_CUDA;
   const int grid = static_cast<int>(std::min<int64_t>(rows, int64_t(num_sms()) * 16));
   k_topk<<<grid, kTopkThreads, smem, s>>>(scores, ld, n_c, rows, topk, kTopkCandCap, n_max, idx,
-                                          cnt);
+                                          cnt, rinfo);
   QSA_CHECK_LAUNCH();
   return QSA_OK;
 }
@@ -271,8 +279,12 @@ qsa_status run_scores_and_topk(const void* q_idx, const void* w, const void* kba
   score_tile_token_starts(h_cu, num_seqs, &starts);
   const int ntiles = static_cast<int>(starts.size()) - 1;
   using C = ScoreCfg<16>;
-  const int smem = std::max(C::kSmemBytes, 116 * 1024);   // one CTA per SM (512 TMEM columns)
-  if (!set_smem(k_index_score<16>, smem)) return QSA_ERR_CUDA;
+  // one CTA per SM (512 TMEM columns); select_mode 1 adds the per-row histograms
+  const int smem = g.fused ? C::kSmemBytesFused : std::max(C::kSmemBytes, 116 * 1024);
+  if (!set_smem(k_index_score<16>, std::max(C::kSmemBytes, 116 * 1024)) ||
+      !set_smem(k_index_score<16, true>, C::kSmemBytesFused))
+    return QSA_ERR_CUDA;
+  int32_t* rinfo = g.fused ? reinterpret_cast<int32_t*>(ws + g.o_rinfo) : nullptr;
   int t = 0;
   while (t < ntiles) {
     int e = t + 1;
@@ -287,12 +299,18 @@ qsa_status run_scores_and_topk(const void* q_idx, const void* w, const void* kba
     a.w = reinterpret_cast<const __nv_bfloat16*>(w);
     a.scores = scores;
     a.ld = g.ld;
+    a.rinfo = rinfo;
+    a.topk = g.topk;
     a.st = dev_status(ws);
-    k_index_score<16><<<e - t, C::kThreads, smem, s>>>(tm_kbar, tm_qidx, a);
+    if (g.fused) {
+      k_index_score<16, true><<<e - t, C::kThreads, smem, s>>>(tm_kbar, tm_qidx, a);
+    } else {
+      k_index_score<16><<<e - t, C::kThreads, smem, s>>>(tm_kbar, tm_qidx, a);
+    }
     QSA_CHECK_LAUNCH();
     const int64_t r0 = starts[t], r1 = starts[e];
     qsa_status st = launch_topk(scores, g.ld, n_c + r0, r1 - r0, g.topk, g.max_nc,
-                                idx + r0 * g.topk, cnt + r0, s);
+                                idx + r0 * g.topk, cnt + r0, s, rinfo);
     if (st != QSA_OK) return st;
     t = e;
   }

@@ -899,7 +899,8 @@ __global__ void __launch_bounds__(kTopkThreads, 4) k_topk(const float* __restric
                                                        const int32_t* __restrict__ n_c, int64_t rows,
                                                        int topk, int cap, int n_max,
                                                        int32_t* __restrict__ idx,
-                                                       int32_t* __restrict__ cnt) {
+                                                       int32_t* __restrict__ cnt,
+                                                       const int32_t* __restrict__ rinfo) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   TopkShared& S = *reinterpret_cast<TopkShared*>(smem_raw);
   uint64_t* c = reinterpret_cast<uint64_t*>(smem_raw + kTopkSharedBytes);
@@ -917,6 +918,16 @@ __global__ void __launch_bounds__(kTopkThreads, 4) k_topk(const float* __restric
       continue;
     }
     const float* src = scores + r * ld;
+    uint32_t b1;
+    int above, in_b1;
+    if (rinfo != nullptr) {
+      // the indexer counted the row's first digit and found its threshold bin (select_mode 1)
+      if (tid == 0) s_cc = 0;
+      b1 = static_cast<uint32_t>(rinfo[4 * r]);
+      above = rinfo[4 * r + 1];
+      in_b1 = rinfo[4 * r + 2];
+      __syncthreads();
+    } else {
     // ---- pass 1: first-digit histogram ----
     clear_bins(S.hist, kTopkBins);
     if (tid == 0) s_cc = 0;
@@ -938,8 +949,8 @@ __global__ void __launch_bounds__(kTopkThreads, 4) k_topk(const float* __restric
         if (i0 + q < n) atomicAdd(&S.hist[float_key(x[q]) >> 20], 1u);
     }
     __syncthreads();
-    int above, in_b1;
-    const uint32_t b1 = static_cast<uint32_t>(topk_find_bin(S, S.hist, kTopkBins, topk, &above, &in_b1));
+    b1 = static_cast<uint32_t>(topk_find_bin(S, S.hist, kTopkBins, topk, &above, &in_b1));
+    }
     if (above + in_b1 > cap) {
       topk_row(src, n, topk, nullptr, out, S);
       if (tid == 0) cnt[r] = topk;

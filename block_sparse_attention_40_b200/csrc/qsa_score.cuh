@@ -42,9 +42,14 @@ struct ScoreCfg {
   static constexpr int kHistOff = kBarOff + kNumBars * 8 + 16;
   static constexpr int kHistBytes = NTOK == 1 ? 4096 * 4 : 0;
   static constexpr int kSmemBytes = kHistOff + kHistBytes + 1024;  // + align slack
+  // prefill with select_mode 1: each token row's first-digit histogram, 4096 16-bit counters
+  // packed in pairs, at kHistOff
+  static constexpr int kRowHistWords = 2048;
+  static constexpr int kSmemBytesFused = kHistOff + NTOK * kRowHistWords * 4 + 1024;
   static constexpr uint32_t kIdesc = idesc_bf16_f32(128, kN, 0, 0);
   static_assert(kCtasPerSm * (kSmemBytes + 1024) <= 228 * 1024, "shared memory per SM");
   static_assert(kCtasPerSm * kTmemCols <= 512, "TMEM columns per SM");
+  static_assert(NTOK != 16 || kSmemBytesFused <= 227 * 1024, "shared memory per CTA");
 };
 
 struct ScoreArgs {
@@ -68,6 +73,11 @@ struct ScoreArgs {
   const int32_t* glen;
   int32_t block0;
   uint32_t* hist;          // [B][4096] first-digit histograms of the scores (zeroed), or null
+  // prefill with select_mode 1: per score row, the first-digit threshold bin of its top-k, as
+  // rinfo[4 r] = bin, [4 r + 1] = keys in higher bins, [4 r + 2] = keys in the bin (rows with
+  // more candidates than the budget; null: not built)
+  int32_t* rinfo;
+  int32_t topk;
   // common
   const __nv_bfloat16* w;  // prefill: [T][16]; decode: [B][16]
   float* scores;
@@ -174,7 +184,10 @@ __device__ __forceinline__ ScoreWork<NTOK> score_work(const ScoreArgs& a) {
   return wk;
 }
 
-template <int NTOK>
+// kRowHist (prefill, select_mode 1): also count each token row's first-digit histogram and
+// find its threshold bin (args.rinfo); a separate instantiation, so the default path carries
+// none of it.
+template <int NTOK, bool kRowHist = false>
 __global__ void __launch_bounds__(ScoreCfg<NTOK>::kThreads, ScoreCfg<NTOK>::kCtasPerSm)
     k_index_score(const __grid_constant__ CUtensorMap tmap_kbar,
                   const __grid_constant__ CUtensorMap tmap_qidx, ScoreArgs args) {
@@ -220,6 +233,12 @@ __global__ void __launch_bounds__(ScoreCfg<NTOK>::kThreads, ScoreCfg<NTOK>::kCta
   uint32_t* sHist = reinterpret_cast<uint32_t*>(smem + C::kHistOff);
   if constexpr (NTOK == 1) {
     for (int i = threadIdx.x; i < 4096; i += blockDim.x) sHist[i] = 0;
+  } else {
+    if constexpr (kRowHist) {
+      uint4* h4 = reinterpret_cast<uint4*>(sHist);
+      for (int i = threadIdx.x; i < NTOK * C::kRowHistWords / 4; i += blockDim.x)
+        h4[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
   }
 
   // weights of the tile's tokens, widened to fp32
@@ -362,8 +381,15 @@ __global__ void __launch_bounds__(ScoreCfg<NTOK>::kThreads, ScoreCfg<NTOK>::kCta
         const bool valid = tok < wk.ntok && blk < (NTOK == 1 ? wk.n_c : pos / kBlock);
         if (valid) {
           float* dst = args.scores + (wk.out_row0 + tok) * args.ld + blk;
-          if constexpr (NTOK == 1) st_global_hint(dst, s, pol_keep);
-          else *dst = s;
+          if constexpr (NTOK == 1) {
+            st_global_hint(dst, s, pol_keep);
+          } else {
+            *dst = s;
+            if constexpr (kRowHist) {   // this row's first-digit histogram (16-bit counters)
+              const uint32_t bin = float_key(s) >> 20;
+              atomicAdd(&sHist[tok * C::kRowHistWords + (bin >> 1)], 1u << ((bin & 1u) << 4));
+            }
+          }
         }
         if constexpr (NTOK == 1) {
           if (args.hist && valid) atomicAdd(&sHist[float_key(s) >> 20], 1u);
@@ -377,6 +403,47 @@ __global__ void __launch_bounds__(ScoreCfg<NTOK>::kThreads, ScoreCfg<NTOK>::kCta
       uint32_t* dst = args.hist + static_cast<int64_t>(wk.out_row0) * 4096;
       for (int i = threadIdx.x; i < 4096; i += blockDim.x)
         if (sHist[i]) atomicAdd(&dst[i], sHist[i]);
+    }
+  } else {
+    // select_mode 1: one warp per token row with more candidates than the budget finds the
+    // row's threshold bin (the one the top-k's first pass would find): lane l sums bins
+    // 4095 - 128 l down to 3968 - 128 l, a warp scan from the top finds the lane whose range
+    // holds the topk-th key, and that lane walks its bins
+    if (kRowHist && !*s_abort && warp < NTOK) {
+      const int tok = warp;
+      const int n = (wk.pos0 + tok) / kBlock;
+      if (tok < wk.ntok && n > args.topk) {   // uniform over the warp
+        const uint32_t* h = sHist + tok * C::kRowHistWords;
+        const int top = 4095 - 128 * lane;   // this lane's bins: top .. top - 127
+        int local = 0;
+#pragma unroll 8
+        for (int wd = 0; wd < 64; ++wd) {
+          const uint32_t v = h[(top >> 1) - wd];
+          local += static_cast<int>((v & 0xffffu) + (v >> 16));
+        }
+        int incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        int running = incl - local;   // keys in the bins above this lane's range
+        if (running < args.topk && incl >= args.topk) {
+          for (int bin = top; bin > top - 128; --bin) {
+            const uint32_t v = h[bin >> 1];
+            const int c = static_cast<int>((bin & 1) ? (v >> 16) : (v & 0xffffu));
+            if (running + c >= args.topk) {
+              int32_t* ri = args.rinfo + (wk.out_row0 + tok) * 4;
+              ri[0] = bin;
+              ri[1] = running;
+              ri[2] = c;
+              ri[3] = n;
+              break;
+            }
+            running += c;
+          }
+        }
+      }
     }
   }
   if (warp == 1) {

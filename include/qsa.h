@@ -96,6 +96,14 @@ typedef struct {
                               undefined.  It exercises the bounded-wait unwind (copies in
                               flight drained, tensor memory freed): a normal call may follow at
                               once.  Other values are refused (QSA_ERR_INVALID_ARG). */
+  int32_t select_mode;     /* prefill selection.  0 (default): the indexer writes each score row
+                              and the top-k reads it twice (a first-digit histogram, then the
+                              candidates).  1: the indexer also counts each row's first-digit
+                              histogram in shared memory and finds its threshold bin, so the
+                              top-k reads each row once (rows of fewer than 65,536 candidate
+                              blocks; longer ones take mode 0).  The same selection either way;
+                              mode 1 measured slower (its shared-memory counting slows the
+                              indexer's epilogue).  Other values: QSA_ERR_INVALID_ARG. */
 } qsa_params;
 
 /* KV cache for decode.  Blocks of 4 tokens are contiguous per (sequence, KV head):

@@ -159,3 +159,25 @@ def test_selection_rows_beyond_65536_blocks():
                            np.arange(262_140, 262_160)])
     rows = np.unique(rows)
     _select_check(p, rows)
+
+
+@pytest.mark.parametrize("name", ["tiny", "8k", "8k_int", "drift"])
+def test_select_mode_1_equals_mode_0(name):
+    # select_mode 1 (the indexer finds each row's threshold bin, the top-k reads each row
+    # once) computes the same scores and the same selection: identical indices, counts and
+    # outputs, bit for bit
+    p = (W.custom_prefill([9000, 2222], topk=512, kind="drift", seed=21) if name == "drift"
+         else W.prefill(name))
+    d = p.to(DEV)
+    res = []
+    for mode in (0, 1):
+        ctx = qsa.Prefill(p.cu_seqlens, DEV, p.topk, select_mode=mode)
+        idx, cnt = ctx.select(d.q_idx, d.k_idx, d.w)
+        out = ctx.run(d.q, d.k, d.v, d.q_idx, d.k_idx, d.w)
+        torch.cuda.synchronize()
+        assert ctx.device_error() == ("QSA_OK", 0)
+        res.append((idx, cnt, out))
+    assert torch.equal(res[0][0], res[1][0]) and torch.equal(res[0][1], res[1][1])
+    assert torch.equal(res[0][2], res[1][2])
+    if name == "tiny":
+        prefill_oracle_check(p, res[1][0], res[1][1], res[1][2], np.arange(256))
