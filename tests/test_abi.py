@@ -50,6 +50,14 @@ def test_workspace_sizes_grow_with_work():
         B.prefill_workspace_size([0, 100], 0)
     with pytest.raises(B.QSAError):
         B.prefill_workspace_size([0, 100], 4096)
+    # select_mode 1 adds each score row's threshold record; other modes are refused
+    assert B.prefill_workspace_size([0, 65536], 512, select_mode=1) > big
+    with pytest.raises(B.QSAError):
+        B.prefill_workspace_size([0, 100], 512, select_mode=2)
+    # rows of 65,536 or more candidates (16-bit counters) take mode 0: no extra workspace
+    long_seq = [0, 4 * 65536 + 8]
+    assert (B.prefill_workspace_size(long_seq, 512, select_mode=1) ==
+            B.prefill_workspace_size(long_seq, 512))
     lib = qsa.load()
     desc = B.CacheDesc(0, 0, 0, 0, 0, 64, 262144)
     n = lib.qsa_decode_workspace_size(ctypes.byref(desc), B._params(512))
