@@ -635,8 +635,9 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
       // are combined once at the end.  All groups take identical rescale decisions.
       // A warp's 32 rows belong to about three tokens: the exponentials of each pair of blocks
       // that none of them attends are skipped (a warp-uniform branch) and its P is left zero,
-      // about half of the union's blocks on long rows.  The masking and the maximum still run
-      // over every key (skipping them too measured no faster).
+      // about half of the union's blocks on long rows.  The block mask is applied once per
+      // block: to the block's maximum, and as an exponent offset of -inf for the blocks the
+      // row's token did not select (a bias added to every key cost 6% more time).
       static_assert(C::kSoftGroups == 2, "prefill softmax assumes two warpgroups");
       constexpr int kSG = C::kSoftGroups;
       constexpr int kCols = 128 / kSG;              // keys (and O dims) per group
@@ -674,33 +675,32 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
   #pragma unroll
           for (int c = 0; c < kCols / 32; ++c) tmem_ld32(ts + kCols * wg + 32 * c, sv + 32 * c);
           tmem_wait_ld();
-          // keys of blocks this row's token did not select -> -inf
-  #pragma unroll
-          for (int u = 0; u < kBlk; ++u) {
-            const float bias = ((mword >> u) & 1u) ? 0.f : -INFINITY;
-  #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              sv[4 * u + kk] = __float_as_uint(__uint_as_float(sv[4 * u + kk]) + bias);
-          }
-          // the own block: hide the tokens after the query (only where it lies)
+          // the own block: hide the tokens after the query (only where it lies).  Selects, not
+          // branches on u == tu: the branches made the compiler spill S to local memory.
           const int tu = tail_u - q * C::kChunkBlocks - kBlk * wg;
           if (__any_sync(0xffffffffu, tu >= 0 && tu < kBlk)) {
   #pragma unroll
             for (int u = 0; u < kBlk; ++u) {
-              if (u == tu) {
-                if (tail_last < 1) sv[4 * u + 1] = __float_as_uint(-INFINITY);
-                if (tail_last < 2) sv[4 * u + 2] = __float_as_uint(-INFINITY);
-                if (tail_last < 3) sv[4 * u + 3] = __float_as_uint(-INFINITY);
-              }
+              const bool own = u == tu;
+              sv[4 * u + 1] = (own && tail_last < 1) ? __float_as_uint(-INFINITY) : sv[4 * u + 1];
+              sv[4 * u + 2] = (own && tail_last < 2) ? __float_as_uint(-INFINITY) : sv[4 * u + 2];
+              sv[4 * u + 3] = (own && tail_last < 3) ? __float_as_uint(-INFINITY) : sv[4 * u + 3];
             }
           }
-          float mxs[8];
+          // each block's maximum, -inf for the blocks this row's token did not select
+          float bm[kBlk];
   #pragma unroll
-          for (int j = 0; j < 8; ++j) mxs[j] = __uint_as_float(sv[j]);
+          for (int u = 0; u < kBlk; ++u) {
+            const float bias = ((mword >> u) & 1u) ? 0.f : -INFINITY;
+            bm[u] = fmaxf(fmaxf(__uint_as_float(sv[4 * u]), __uint_as_float(sv[4 * u + 1])),
+                          fmaxf(__uint_as_float(sv[4 * u + 2]), __uint_as_float(sv[4 * u + 3]))) + bias;
+          }
+          static_assert(kBlk == 16, "a four-level tree");
   #pragma unroll
-          for (int j = 8; j < kCols; ++j) mxs[j & 7] = fmaxf(mxs[j & 7], __uint_as_float(sv[j]));
-          mx = fmaxf(fmaxf(fmaxf(mxs[0], mxs[1]), fmaxf(mxs[2], mxs[3])),
-                     fmaxf(fmaxf(mxs[4], mxs[5]), fmaxf(mxs[6], mxs[7])));
+          for (int u = 0; u < 8; ++u) bm[u] = fmaxf(bm[u], bm[u + 8]);
+  #pragma unroll
+          for (int u = 0; u < 4; ++u) bm[u] = fmaxf(bm[u], bm[u + 4]);
+          mx = fmaxf(fmaxf(bm[0], bm[2]), fmaxf(bm[1], bm[3]));
         }
         // exchange the partial row maxima (every softmax warp takes part, active or not)
         xmax[(b * kSG + wg) * 128 + row] = mx;
@@ -729,8 +729,10 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
   #pragma unroll
               for (int jj = 0; jj < 2 * kSk; ++jj) {
                 const int j = gi * 2 * kSk + jj;
-                const float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * j]), sl2, mneg));
-                const float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * j + 1]), sl2, mneg));
+                // blocks the row's token did not select: exponent -inf, so P = 0
+                const float off = ((mword >> (j >> 1)) & 1u) ? mneg : -INFINITY;
+                const float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * j]), sl2, off));
+                const float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * j + 1]), sl2, off));
                 lsum[j & 3] += p0 + p1;
                 sv[j] = pack_bf16x2(p0, p1);
               }
