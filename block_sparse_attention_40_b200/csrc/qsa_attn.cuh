@@ -711,7 +711,9 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
   #pragma unroll
           for (int o = 1; o < kSG; ++o) mx = fmaxf(mx, xmax[(b * kSG + ((wg + o) % kSG)) * 128 + row]);
           const float m_cand = fmaxf(m, mx * sl2);
-          const bool grow = m_cand > m + 8.f || (m == -INFINITY && m_cand > -INFINITY);
+          // lazy rescale: P may reach 2^16 (bf16 keeps its relative precision; O and the sum are
+          // fp32), so O is rescaled only when a row's maximum grows by more than 16 (log2 units)
+          const bool grow = m_cand > m + 16.f || (m == -INFINITY && m_cand > -INFINITY);
           const bool rescale = __any_sync(0xffffffffu, grow);
           float alpha = 1.f;
           if (rescale) {
