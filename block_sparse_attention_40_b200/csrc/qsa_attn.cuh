@@ -66,7 +66,9 @@ struct AttnCfg {
   static constexpr int kXBytes = (2 * kSoftGroups * 128 + kSoftGroups * 128) * 4;
   static constexpr int kBarOff = kXOff + kXBytes;
   static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 1 + 1 + 1;
-  static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
+  // the block-mask bias table: entry n holds, for bits 0..3 of n, 0 (block selected) or -inf
+  static constexpr int kLutOff = (kBarOff + kNumBars * 8 + 16 + 15) / 16 * 16;   // 16 x float4
+  static constexpr int kSmemBytes = kLutOff + 256 + 1024;
   static constexpr int kTmemCols = 512;   // S0 [0,128) S1 [128,256) O [256,384)
   static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0, 0);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 0, 1);   // B = V is MN-major
@@ -318,6 +320,9 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
     *s_abort = 0;
     fence_mbar_init();
   }
+  if (threadIdx.x < 64)
+    reinterpret_cast<float*>(smem + C::kLutOff)[threadIdx.x] =
+        (((threadIdx.x >> 2) >> (threadIdx.x & 3)) & 1u) ? 0.f : -INFINITY;
   // zero the rows of Q that TMA never writes: rows 12R..127 (prefill), or rows 32q+12..32q+31
   // of every lane quarter q (decode: the 12 head rows are loaded at rows 32q..32q+11)
   {
@@ -345,7 +350,7 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
   const uint32_t* masks = reinterpret_cast<const uint32_t*>(rec + args.pl.mask_off());
   const int mwords = args.pl.umax / 32;
   const int col0 = kDec ? 0 : g * kHeadDim;
-  // P: written over S in prefill; in its own columns [384, 512) in decode
+  // P: its own columns [384, 512), two buffers of 64 (bf16 pairs)
   const uint32_t tmem_P = tmem + 384;
   constexpr int kPStride = 64;
 
@@ -637,7 +642,8 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
       // that none of them attends are skipped (a warp-uniform branch) and its P is left zero,
       // about half of the union's blocks on long rows.  The block mask is applied once per
       // block: to the block's maximum, and as an exponent offset of -inf for the blocks the
-      // row's token did not select (a bias added to every key cost 6% more time).
+      // row's token did not select (a bias added to every key cost 6% more time).  The softmax
+      // is bound by its instruction stream: every instruction taken out of a chunk shows.
       static_assert(C::kSoftGroups == 2, "prefill softmax assumes two warpgroups");
       constexpr int kSG = C::kSoftGroups;
       constexpr int kCols = 128 / kSG;              // keys (and O dims) per group
@@ -658,6 +664,7 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
       const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
       const uint32_t* mrow = masks + tr * mwords;
       uint32_t mword_next = row_ok ? mrow[c_begin] : 0u;
+      const float4* lut4 = reinterpret_cast<const float4*>(smem + C::kLutOff);
       bool ok = true;
       for (int i = 0; i < nchunks; ++i) {
         const int b = i & 1;
@@ -671,6 +678,14 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
         uint32_t sv[kCols];
         const uint32_t ts = tmem + lane_base + b * 128;
         float mx = -INFINITY;
+        // 0 / -inf per block of this row's token, four blocks per table read (a bit test and a
+        // select per block cost 1.7% more time)
+        float bias[kBlk];
+  #pragma unroll
+        for (int n = 0; n < kBlk / 4; ++n) {
+          const float4 bb = lut4[(mword >> (4 * n)) & 15u];
+          bias[4 * n] = bb.x; bias[4 * n + 1] = bb.y; bias[4 * n + 2] = bb.z; bias[4 * n + 3] = bb.w;
+        }
         if (ok && warp_active) {
   #pragma unroll
           for (int c = 0; c < kCols / 32; ++c) tmem_ld32(ts + kCols * wg + 32 * c, sv + 32 * c);
@@ -691,9 +706,8 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
           float bm[kBlk];
   #pragma unroll
           for (int u = 0; u < kBlk; ++u) {
-            const float bias = ((mword >> u) & 1u) ? 0.f : -INFINITY;
             bm[u] = fmaxf(fmaxf(__uint_as_float(sv[4 * u]), __uint_as_float(sv[4 * u + 1])),
-                          fmaxf(__uint_as_float(sv[4 * u + 2]), __uint_as_float(sv[4 * u + 3]))) + bias;
+                          fmaxf(__uint_as_float(sv[4 * u + 2]), __uint_as_float(sv[4 * u + 3]))) + bias[u];
           }
           static_assert(kBlk == 16, "a four-level tree");
   #pragma unroll
@@ -723,7 +737,7 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
           const float mneg = (m == -INFINITY) ? 0.f : -m;
           // P overwrites S in registers: packed pair j lands in sv[j], whose S value (key j) was
           // consumed at pair j/2 <= j
-          float lsum[4] = {0.f, 0.f, 0.f, 0.f};
+          uint64_t lsum2[2] = {0ull, 0ull};   // row sums as packed pairs (add.rn.f32x2)
           constexpr int kSk = 2;                 // blocks per skip decision (1, 2, 4: 2 measured best)
   #pragma unroll
           for (int gi = 0; gi < kBlk / kSk; ++gi) {
@@ -732,10 +746,10 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
               for (int jj = 0; jj < 2 * kSk; ++jj) {
                 const int j = gi * 2 * kSk + jj;
                 // blocks the row's token did not select: exponent -inf, so P = 0
-                const float off = ((mword >> (j >> 1)) & 1u) ? mneg : -INFINITY;
+                const float off = mneg + bias[j >> 1];
                 const float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * j]), sl2, off));
                 const float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * j + 1]), sl2, off));
-                lsum[j & 3] += p0 + p1;
+                lsum2[j & 1] = f2_add(lsum2[j & 1], f2_pack(p0, p1));
                 sv[j] = pack_bf16x2(p0, p1);
               }
             } else {
@@ -743,7 +757,8 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
               for (int jj = 0; jj < 2 * kSk; ++jj) sv[gi * 2 * kSk + jj] = 0u;
             }
           }
-          l = l * alpha + ((lsum[0] + lsum[1]) + (lsum[2] + lsum[3]));
+          const uint64_t ls = f2_add(lsum2[0], lsum2[1]);
+          l = l * alpha + (f2_lo(ls) + f2_hi(ls));
           // packed P of my keys -> columns kCols/2 sg .. of this buffer's P (P.V of chunk i-2,
           // which last read them, completed before S_i: one commit tracks every earlier MMA)
           tmem_st32(tmem_P + lane_base + b * kPStride + 32 * wg, sv);
