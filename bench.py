@@ -42,18 +42,18 @@ DEC_BATCH, DEC_CAP = 64, 262144
 # figure is reported only while the sources are unchanged; otherwise the roofline's
 # "traffic" is null until a new capture is taken.
 NCU_TRAFFIC = {
-    # 313,253,376 B read + 175,233,280 B written by one 32K-token prefill attention launch
+    # 313,251,072 B read + 175,057,920 B written by one 32K-token prefill attention launch
     # (profiles/k_sparse_attn_prefill_32k.md), per token; the attention's bytes (Q, O, the
     # gathered K/V tiles, the plan) grow with the tokens of the launch.
-    "prefill_attention": (488486656 / 32768,
-                          "6fd5987da9b29cdf76ac210495674403251e61da9f46aa27f1e7a8ecc8ebace1",
+    "prefill_attention": (488308992 / 32768,
+                          "c1aa23be1a9debf2fe6d8e831ea38176624c4ffdbca4c4ea2f1490f9c2039d3f",
                           "ncu dram__bytes_read.sum + dram__bytes_write.sum of one 32K-token "
                           "launch (profiles/k_sparse_attn_prefill_32k.md), scaled by tokens"),
     # The seven kernels of one 256K x 64 decode step, one ncu capture each (1 pass): reads
-    # 690,889,984 B, writes 6,281,216 B (profiles/decode_step_dram_decode256k_b64.md); per
+    # 690,877,696 B, writes 6,285,824 B (profiles/decode_step_dram_decode256k_b64.md); per
     # sequence of the batch.
-    "decode_step": (697171200 / 64,
-                    "3b817e0534621b30677800f9def2c8202e5f249268f3373c45a05b69e0dcf0e6",
+    "decode_step": (697163520 / 64,
+                    "4b70f46519a745f3e0ed12920e76c5b02414030c20fe2ecbf6731d3baebf6410",
                     "ncu dram__bytes_read.sum + dram__bytes_write.sum of the seven kernels of "
                     "one 256K x 64 decode step (profiles/decode_step_dram_decode256k_b64.md)"),
 }
