@@ -42,18 +42,18 @@ DEC_BATCH, DEC_CAP = 64, 262144
 # figure is reported only while the sources are unchanged; otherwise the roofline's
 # "traffic" is null until a new capture is taken.
 NCU_TRAFFIC = {
-    # 313,251,072 B read + 175,057,920 B written by one 32K-token prefill attention launch
+    # 312,955,904 B read + 175,307,008 B written by one 32K-token prefill attention launch
     # (profiles/k_sparse_attn_prefill_32k.md), per token; the attention's bytes (Q, O, the
     # gathered K/V tiles, the plan) grow with the tokens of the launch.
-    "prefill_attention": (488308992 / 32768,
-                          "c1aa23be1a9debf2fe6d8e831ea38176624c4ffdbca4c4ea2f1490f9c2039d3f",
+    "prefill_attention": (488262912 / 32768,
+                          "2a4604d3d88ad5c9ad4d4f32dc0944e48f64cdb3eeb59af5b2e3aa667291549a",
                           "ncu dram__bytes_read.sum + dram__bytes_write.sum of one 32K-token "
                           "launch (profiles/k_sparse_attn_prefill_32k.md), scaled by tokens"),
     # The seven kernels of one 256K x 64 decode step, one ncu capture each (1 pass): reads
-    # 690,877,696 B, writes 6,285,824 B (profiles/decode_step_dram_decode256k_b64.md); per
+    # 690,883,840 B, writes 6,260,224 B (profiles/decode_step_dram_decode256k_b64.md); per
     # sequence of the batch.
-    "decode_step": (697163520 / 64,
-                    "4b70f46519a745f3e0ed12920e76c5b02414030c20fe2ecbf6731d3baebf6410",
+    "decode_step": (697144064 / 64,
+                    "9b869a4aa4619bff4dc4b0732644259399682afa8f5f8a368e55b5e03fe3bb19",
                     "ncu dram__bytes_read.sum + dram__bytes_write.sum of the seven kernels of "
                     "one 256K x 64 decode step (profiles/decode_step_dram_decode256k_b64.md)"),
 }
