@@ -394,6 +394,9 @@ QSA_API qsa_status qsa_decode_paged(const void *q, const qsa_paged_cache *cache,
  *     S_t = alpha_t S_{t-1} + beta_t (v_t - alpha_t S_{t-1} k_t) k_t^T,    o_t = S_t q_t
  * with alpha_t = exp(log_alpha_t).  q and k are used as given (any normalisation or scaling
  * happens before the call); log_alpha below -87 counts as -87 (a full reset, to fp32 range).
+ * Arithmetic: the chunked products run on the tensor cores with TF32 operands and fp32
+ * accumulation; the operands that carry into the state are split into two TF32 parts (about
+ * fp32 accuracy); the state is fp32.
  *   q, k, v      bf16 [T][heads][128], 16-byte aligned
  *   log_alpha    fp32 [T][heads] (<= 0 keeps the state bounded), beta fp32 [T][heads]
  *   d_cu_seqlens int32 [num_seqs+1] on the device, h_cu_seqlens the same on the host
