@@ -46,14 +46,14 @@ NCU_TRAFFIC = {
     # (profiles/k_sparse_attn_prefill_32k.md), per token; the attention's bytes (Q, O, the
     # gathered K/V tiles, the plan) grow with the tokens of the launch.
     "prefill_attention": (488262912 / 32768,
-                          "2a4604d3d88ad5c9ad4d4f32dc0944e48f64cdb3eeb59af5b2e3aa667291549a",
+                          "d1ea05a60e832f72204bcec12ba314564f4d847fe9118e6a990904e7bda79a7d",
                           "ncu dram__bytes_read.sum + dram__bytes_write.sum of one 32K-token "
                           "launch (profiles/k_sparse_attn_prefill_32k.md), scaled by tokens"),
     # The seven kernels of one 256K x 64 decode step, one ncu capture each (1 pass): reads
     # 690,883,840 B, writes 6,260,224 B (profiles/decode_step_dram_decode256k_b64.md); per
     # sequence of the batch.
     "decode_step": (697144064 / 64,
-                    "9b869a4aa4619bff4dc4b0732644259399682afa8f5f8a368e55b5e03fe3bb19",
+                    "d6c1add7fa73aec5ec5dec7604922821ea7d8e2788d833d5ac7373ea6323d38b",
                     "ncu dram__bytes_read.sum + dram__bytes_write.sum of the seven kernels of "
                     "one 256K x 64 decode step (profiles/decode_step_dram_decode256k_b64.md)"),
 }

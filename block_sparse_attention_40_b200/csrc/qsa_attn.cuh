@@ -637,14 +637,15 @@ __global__ void __launch_bounds__(AttnCfg::kThreads, 1)
       // kSoftGroups warpgroups share each row: group sg handles keys [kCols sg, kCols (sg + 1))
       // of every chunk and dims [kCols sg, ...) of O.  Row maxima are exchanged through shared
       // memory (double-buffered by chunk parity, one named barrier per chunk and lane quarter,
-      // ids 2..5); partial row sums
-      // are combined once at the end.  All groups take identical rescale decisions.
+      // ids 2..5); partial row sums are combined once at the end.  All groups take identical
+      // rescale decisions.
       // A warp's 32 rows belong to about three tokens: the exponentials of each pair of blocks
       // that none of them attends are skipped (a warp-uniform branch) and its P is left zero,
       // about half of the union's blocks on long rows.  The block mask is applied once per
       // block: to the block's maximum, and as an exponent offset of -inf for the blocks the
       // row's token did not select (a bias added to every key cost 6% more time).  The softmax
-      // is bound by its instruction stream: every instruction taken out of a chunk shows.
+      // is bound mostly by its instruction stream: most instructions taken out of a chunk
+      // showed in the kernel's time.
       static_assert(C::kSoftGroups == 2, "prefill softmax assumes two warpgroups");
       constexpr int kSG = C::kSoftGroups;
       constexpr int kCols = 128 / kSG;              // keys (and O dims) per group
